@@ -1,0 +1,123 @@
+// Weighted combine: the MoE block's final floating-point reduction.
+//
+// "DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 3 ("Final Reduction Is
+// The Core Drift Point"): the order, dtype and downcast point of the combine are the
+// contract. "From Expert Reduction to Behavioral Divergence" (arXiv 2607.28097, Abstract):
+// different orders of the expert sum are observably different, so one order is fixed:
+// rank order 0..K-1, each product w_j * y rounded to fp32, sequential fp32 adds, the
+// shared expert added last, one bf16 round-to-nearest-even at the end. No FMA, no atomics;
+// every output element is produced by exactly one thread.
+//
+// Memory-bound: each thread owns 8 consecutive columns (one 16-byte vector) of a token,
+// issues the K row loads first (K independent 128-bit loads in flight), then reduces in
+// rank order and writes one 128-bit vector.
+#include <cuda_bf16.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b)
+{
+    const __nv_bfloat16 x = __float2bfloat16_rn(a), y = __float2bfloat16_rn(b);
+    return (uint32_t)__bfloat16_as_ushort(x) | ((uint32_t)__bfloat16_as_ushort(y) << 16);
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
+                                                      const float* __restrict__ w,
+                                                      const int32_t* __restrict__ dest_row,
+                                                      const uint4* __restrict__ y_shared,
+                                                      const uint8_t* __restrict__ mask, int T,
+                                                      int K, int vec_per_row,
+                                                      uint4* __restrict__ out)
+{
+    const int64_t total = (int64_t)T * vec_per_row;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = idx / vec_per_row;
+        const int v = (int)(idx - t * vec_per_row);
+        if (mask != nullptr && mask[t] == 0) {
+            out[idx] = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        uint4 rows[KMAX];
+        float wj[KMAX];
+        int32_t dr[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < K) {
+                dr[j] = dest_row[t * K + j];
+                wj[j] = w[t * K + j];
+                rows[j] = (dr[j] >= 0) ? y[(int64_t)dr[j] * vec_per_row + v]
+                                       : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        float acc[8];
+        bool first = true;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < K && dr[j] >= 0) {
+                const uint32_t q[4] = {rows[j].x, rows[j].y, rows[j].z, rows[j].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float p0 = __fmul_rn(wj[j], bf16_lo(q[c]));
+                    const float p1 = __fmul_rn(wj[j], bf16_hi(q[c]));
+                    acc[2 * c] = first ? p0 : __fadd_rn(acc[2 * c], p0);
+                    acc[2 * c + 1] = first ? p1 : __fadd_rn(acc[2 * c + 1], p1);
+                }
+                first = false;
+            }
+        }
+        if (first) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+        }
+        if (y_shared != nullptr) {
+            const uint4 s = y_shared[idx];
+            const uint32_t q[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                acc[2 * c] = __fadd_rn(acc[2 * c], bf16_lo(q[c]));
+                acc[2 * c + 1] = __fadd_rn(acc[2 * c + 1], bf16_hi(q[c]));
+            }
+        }
+        out[idx] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                              pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+    }
+}
+
+template <int KMAX>
+cudaError_t launch_k(const moe_cfg& c, const uint16_t* y, const float* w, const int32_t* dr,
+                     const uint16_t* ys, const uint8_t* mask, uint16_t* out, cudaStream_t st)
+{
+    const int vec = c.H / 8;
+    const int64_t total = (int64_t)c.T * vec;
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    combine_kernel<KMAX><<<(unsigned)blocks, 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys), mask,
+        c.T, c.K, vec, reinterpret_cast<uint4*>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
+                           const int32_t* dest_row, const uint16_t* y_shared,
+                           const uint8_t* mask, uint16_t* out, cudaStream_t st)
+{
+    if (c.T == 0) return cudaSuccess;
+    if (c.K <= 1) return launch_k<1>(c, y, w, dest_row, y_shared, mask, out, st);
+    if (c.K <= 2) return launch_k<2>(c, y, w, dest_row, y_shared, mask, out, st);
+    if (c.K <= 4) return launch_k<4>(c, y, w, dest_row, y_shared, mask, out, st);
+    if (c.K <= 8) return launch_k<8>(c, y, w, dest_row, y_shared, mask, out, st);
+    return launch_k<16>(c, y, w, dest_row, y_shared, mask, out, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,391 @@
+// C ABI of libmoe_b200 (declared in include/moe.h): argument checks, workspace layout,
+// tensor-core GEMM set-up and the launch sequence of each boundary. Host code only; the
+// kernels live in route.cu, permute.cu, tc_gemm.cu and combine.cu.
+#include <math.h>
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+int num_sms()
+{
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+bool device_is_sm100()
+{
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return false;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return false;
+    return major == 10 && minor == 0;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+int check_cfg(const moe_cfg* c)
+{
+    if (c == nullptr) return MOE_ERR_ARG;
+    if (c->T < 0 || c->E < 1 || c->E > 1024 || c->K < 1 || c->K > 16 || c->K > c->E)
+        return MOE_ERR_SHAPE;
+    if (c->H < 128 || c->H > 16384 || c->H % 128 != 0) return MOE_ERR_SHAPE;
+    if (c->I < 128 || c->I > 16384 || c->I % 128 != 0) return MOE_ERR_SHAPE;
+    if (c->I_shared < 0 || c->I_shared > 32768 || c->I_shared % 128 != 0) return MOE_ERR_SHAPE;
+    if ((int64_t)c->T * c->K >= ((int64_t)1 << 31)) return MOE_ERR_SHAPE;
+    if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_SHAPE;
+    if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_SHAPE;
+    if (!isfinite(c->route_scale)) return MOE_ERR_SHAPE;
+    return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device()
+{
+    return device_is_sm100() ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// scratch of moe_grouped_ffn: h [T*K, I] (+ h_shared [T, I_shared]), bf16
+struct FfnLayout {
+    size_t h, h_s, total;
+};
+
+FfnLayout ffn_layout(const moe_cfg& c)
+{
+    FfnLayout L{};
+    const size_t A = (size_t)c.T * c.K;
+    size_t off = 0;
+    L.h = off;
+    off += up(A * c.I * 2);
+    L.h_s = off;
+    off += up((size_t)c.T * c.I_shared * 2);
+    L.total = off;
+    return L;
+}
+
+// scratch of moe_forward
+struct FwdLayout {
+    size_t logits, ids, w, offsets, perm_token, dest_row, perm_ws, x_perm, y, y_s, ffn, total;
+};
+
+FwdLayout fwd_layout(const moe_cfg& c)
+{
+    FwdLayout L{};
+    const size_t A = (size_t)c.T * c.K;
+    size_t off = 0;
+    L.logits = off;     off += up((size_t)c.T * c.E * 4);
+    L.ids = off;        off += up(A * 4);
+    L.w = off;          off += up(A * 4);
+    L.offsets = off;    off += up((size_t)(c.E + 1) * 4);
+    L.perm_token = off; off += up(A * 4);
+    L.dest_row = off;   off += up(A * 4);
+    L.perm_ws = off;    off += up(permute_ws_bytes(c));
+    L.x_perm = off;     off += up(A * c.H * 2);
+    L.y = off;          off += up(A * c.H * 2);
+    L.y_s = off;        off += up(c.I_shared ? (size_t)c.T * c.H * 2 : 0);
+    L.ffn = off;        off += ffn_layout(c).total;
+    L.total = off;
+    return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off)
+{
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int rec(void* const* ev, int i, cudaStream_t st)
+{
+    if (ev == nullptr || ev[i] == nullptr) return MOE_OK;
+    return cuda_rc(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st));
+}
+
+// router logits on the tensor cores: logits[T,E] = x . Wr^T (+ bias), fp32
+cudaError_t router_logits(const moe_cfg& c, const uint16_t* x, const uint16_t* wr,
+                          const float* logit_bias, float* logits, int32_t* status,
+                          cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_F32;
+    p.a = x;
+    p.a_rows = c.T;
+    p.b = wr;
+    p.b_rows_per_group = c.E;
+    p.k = c.H;
+    p.n = c.E;
+    p.groups = 1;
+    p.offsets = nullptr;
+    p.rows = c.T;
+    p.out = logits;
+    p.ldo = c.E;
+    p.bias = logit_bias;
+    p.status = status;
+    return launch_tc_gemm(p, st);
+}
+
+// gate_up + SwiGLU over grouped rows: h[r] = silu(a_r . W1g^T) * (a_r . W1u^T)
+cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                    int rows, const uint16_t* w13, int H, int I, uint16_t* h, int32_t* status,
+                    cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_SWIGLU;
+    p.a = a;
+    p.a_rows = a_rows;
+    p.b = w13;
+    p.b_rows_per_group = 2 * I;
+    p.k = H;
+    p.n = I;
+    p.groups = groups;
+    p.offsets = offsets;
+    p.rows = rows;
+    p.out = h;
+    p.ldo = I;
+    p.status = status;
+    return launch_tc_gemm(p, st);
+}
+
+// down over grouped rows: y[r] = h_r . W2^T
+cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int groups, int rows,
+                 const uint16_t* w2, int H, int I, uint16_t* y, int32_t* status, cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_BF16;
+    p.a = h;
+    p.a_rows = a_rows;
+    p.b = w2;
+    p.b_rows_per_group = H;
+    p.k = I;
+    p.n = H;
+    p.groups = groups;
+    p.offsets = offsets;
+    p.rows = rows;
+    p.out = y;
+    p.ldo = H;
+    p.status = status;
+    return launch_tc_gemm(p, st);
+}
+
+int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm, const int32_t* offsets,
+             const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s, const uint16_t* w2_s,
+             uint16_t* y, uint16_t* y_shared, int32_t* status, void* ws, void* const* ev,
+             cudaStream_t st)
+{
+    const FfnLayout L = ffn_layout(c);
+    const int64_t A = (int64_t)c.T * c.K;
+    uint16_t* h = at<uint16_t>(ws, L.h);
+    int rc = cuda_rc(gate_up(x_perm, A, offsets, c.E, 0, w13, c.H, c.I, h, status, st));
+    if (rc != MOE_OK) return rc;
+    if ((rc = rec(ev, 4, st)) != MOE_OK) return rc;
+    rc = cuda_rc(down(h, A, offsets, c.E, 0, w2, c.H, c.I, y, status, st));
+    if (rc != MOE_OK) return rc;
+    if ((rc = rec(ev, 5, st)) != MOE_OK) return rc;
+    if (c.I_shared > 0 && w13_s != nullptr) {
+        uint16_t* h_s = at<uint16_t>(ws, L.h_s);
+        rc = cuda_rc(gate_up(x, c.T, nullptr, 1, c.T, w13_s, c.H, c.I_shared, h_s, status, st));
+        if (rc != MOE_OK) return rc;
+        rc = cuda_rc(down(h_s, c.T, nullptr, 1, c.T, w2_s, c.H, c.I_shared, y_shared, status, st));
+        if (rc != MOE_OK) return rc;
+    }
+    return rec(ev, 6, st);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+MOE_API int moe_abi_version(void) { return 100; }
+
+MOE_API const char* moe_status_string(int code)
+{
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument (null or misaligned pointer)";
+        case MOE_ERR_SHAPE: return "unsupported shape or configuration";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case MOE_ERR_UNIMPLEMENTED: return "not implemented in this build";
+        case MOE_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
+        default: return "unknown status";
+    }
+}
+
+MOE_API size_t moe_workspace_bytes(const moe_cfg* cfg, int stage)
+{
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    switch (stage) {
+        case MOE_STAGE_ROUTE: return 0;
+        case MOE_STAGE_PERMUTE: return permute_ws_bytes(*cfg);
+        case MOE_STAGE_FFN: return ffn_layout(*cfg).total;
+        case MOE_STAGE_COMBINE: return 0;
+        case MOE_STAGE_FORWARD: return fwd_layout(*cfg).total;
+        default: return 0;
+    }
+}
+
+MOE_API int moe_route(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                      const float* logit_bias, const float* sel_bias, const uint8_t* token_mask,
+                      float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                      void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_ARG;
+    if (x != nullptr && (w_router == nullptr || !aligned16(x) || !aligned16(w_router)))
+        return MOE_ERR_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
+        return rc;
+    if (x != nullptr) {
+        rc = cuda_rc(router_logits(*cfg, x, w_router, logit_bias, logits, status, st));
+        if (rc != MOE_OK) return rc;
+    }
+    return cuda_rc(launch_route(*cfg, logits, sel_bias, token_mask, topk_ids, topk_w, status, st));
+}
+
+MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint16_t* x,
+                        int32_t* offsets, int32_t* perm_token, int32_t* dest_row,
+                        uint16_t* x_perm, int32_t* status, void* ws, size_t ws_bytes,
+                        void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (topk_ids == nullptr || offsets == nullptr || perm_token == nullptr || dest_row == nullptr)
+        return MOE_ERR_ARG;
+    if (x_perm != nullptr && (x == nullptr || !aligned16(x) || !aligned16(x_perm)))
+        return MOE_ERR_ARG;
+    if (ws_bytes < permute_ws_bytes(*cfg) || ws == nullptr) return MOE_ERR_WORKSPACE;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
+        return rc;
+    rc = cuda_rc(launch_permute(*cfg, topk_ids, offsets, perm_token, dest_row, status, ws, st));
+    if (rc != MOE_OK || x_perm == nullptr) return rc;
+    return cuda_rc(launch_gather_rows(*cfg, x, perm_token, offsets, x_perm, st));
+}
+
+MOE_API int moe_grouped_ffn(const moe_cfg* cfg, const uint16_t* x, const uint16_t* x_perm,
+                            const int32_t* perm_token, const int32_t* offsets,
+                            const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
+                            const uint16_t* w2_s, uint16_t* y, uint16_t* y_shared,
+                            int32_t* status, void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (offsets == nullptr || w13 == nullptr || w2 == nullptr || y == nullptr) return MOE_ERR_ARG;
+    if (!aligned16(w13) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_ARG;
+    const bool shared = cfg->I_shared > 0;
+    if (shared && (x == nullptr || w13_s == nullptr || w2_s == nullptr || y_shared == nullptr ||
+                   !aligned16(x) || !aligned16(w13_s) || !aligned16(w2_s) || !aligned16(y_shared)))
+        return MOE_ERR_ARG;
+    if (x_perm == nullptr) {
+        if (perm_token == nullptr || x == nullptr) return MOE_ERR_ARG;
+        return MOE_ERR_UNIMPLEMENTED;
+    }
+    if (!aligned16(x_perm)) return MOE_ERR_ARG;
+    if (ws == nullptr || ws_bytes < ffn_layout(*cfg).total) return MOE_ERR_WORKSPACE;
+    if (cfg->T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
+        return rc;
+    return ffn_impl(*cfg, x, x_perm, offsets, w13, w2, shared ? w13_s : nullptr,
+                    shared ? w2_s : nullptr, y, y_shared, status, ws, nullptr, st);
+}
+
+MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* y, const float* topk_w,
+                        const int32_t* dest_row, const uint16_t* y_shared,
+                        const uint8_t* token_mask, uint16_t* out, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (y == nullptr || topk_w == nullptr || dest_row == nullptr || out == nullptr)
+        return MOE_ERR_ARG;
+    if (!aligned16(y) || !aligned16(out) || (y_shared != nullptr && !aligned16(y_shared)))
+        return MOE_ERR_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    return cuda_rc(launch_combine(*cfg, y, topk_w, dest_row, y_shared, token_mask, out,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                        const float* logit_bias, const float* sel_bias, const uint8_t* token_mask,
+                        const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
+                        const uint16_t* w2_s, uint16_t* out, float* logits, int32_t* topk_ids,
+                        float* topk_w, int32_t* offsets, int32_t* status, void* ws,
+                        size_t ws_bytes, void* const* stage_events, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    const moe_cfg& c = *cfg;
+    if (x == nullptr || w_router == nullptr || w13 == nullptr || w2 == nullptr || out == nullptr ||
+        status == nullptr)
+        return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) ||
+        !aligned16(out))
+        return MOE_ERR_ARG;
+    const bool shared = c.I_shared > 0;
+    if (shared && (w13_s == nullptr || w2_s == nullptr || !aligned16(w13_s) || !aligned16(w2_s)))
+        return MOE_ERR_ARG;
+    const FwdLayout L = fwd_layout(c);
+    if (ws == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (c.T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* const* ev = stage_events;
+
+    float* lg = logits ? logits : at<float>(ws, L.logits);
+    int32_t* ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
+    float* w = topk_w ? topk_w : at<float>(ws, L.w);
+    int32_t* offs = offsets ? offsets : at<int32_t>(ws, L.offsets);
+    int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t* dest_row = at<int32_t>(ws, L.dest_row);
+    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+    uint16_t* y = at<uint16_t>(ws, L.y);
+    uint16_t* y_s = shared ? at<uint16_t>(ws, L.y_s) : nullptr;
+
+    if ((rc = rec(ev, 0, st)) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(router_logits(c, x, w_router, logit_bias, lg, status, st))) != MOE_OK)
+        return rc;
+    if ((rc = rec(ev, 1, st)) != MOE_OK) return rc;
+    if ((rc = cuda_rc(launch_route(c, lg, sel_bias, token_mask, ids, w, status, st))) != MOE_OK)
+        return rc;
+    if ((rc = rec(ev, 2, st)) != MOE_OK) return rc;
+    rc = cuda_rc(launch_permute(c, ids, offs, perm_token, dest_row, status,
+                                at<void>(ws, L.perm_ws), st));
+    if (rc != MOE_OK) return rc;
+    if ((rc = cuda_rc(launch_gather_rows(c, x, perm_token, offs, x_perm, st))) != MOE_OK) return rc;
+    if ((rc = rec(ev, 3, st)) != MOE_OK) return rc;
+    rc = ffn_impl(c, x, x_perm, offs, w13, w2, shared ? w13_s : nullptr, shared ? w2_s : nullptr,
+                  y, y_s, status, at<void>(ws, L.ffn), ev, st);
+    if (rc != MOE_OK) return rc;
+    rc = cuda_rc(launch_combine(c, y, w, dest_row, y_s, token_mask, out, st));
+    if (rc != MOE_OK) return rc;
+    return rec(ev, 7, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// Internal declarations shared by the CUDA translation units of libmoe_b200.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ status helpers
+
+__device__ __forceinline__ void status_add(int32_t* status, int word, int v)
+{
+    if (status != nullptr && v != 0) atomicAdd(status + word, v);
+}
+
+// ------------------------------------------------------------------ launchers
+
+// routing: one warp per token
+cudaError_t launch_route(const moe_cfg& c, const float* logits, const float* sel_bias,
+                         const uint8_t* mask, int32_t* ids, float* w, int32_t* status,
+                         cudaStream_t st);
+
+// dispatch
+size_t permute_ws_bytes(const moe_cfg& c);
+cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offsets,
+                           int32_t* perm_token, int32_t* dest_row, int32_t* status, void* ws,
+                           cudaStream_t st);
+cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* perm_token,
+                               const int32_t* offsets, uint16_t* x_perm, cudaStream_t st);
+
+// combine
+cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
+                           const int32_t* dest_row, const uint16_t* y_shared,
+                           const uint8_t* mask, uint16_t* out, cudaStream_t st);
+
+// tensor-core GEMMs (tcgen05 / TMEM / TMA)
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_F32 = 2 };
+
+struct GemmProblem {
+    int epilogue;            // GemmEpilogue
+    const uint16_t* a;       // A [a_rows, k] bf16 (row-major, K-major)
+    int64_t a_rows;          // rows of the A buffer (TMA bound)
+    const uint16_t* b;       // B [groups * b_rows_per_group, k] bf16
+    int b_rows_per_group;    // SWIGLU: 2*I (gate rows then up rows); else N
+    int k;                   // reduction length (multiple of 64)
+    int n;                   // output columns per group (SWIGLU: I)
+    int groups;              // number of row groups (experts)
+    const int32_t* offsets;  // device [groups+1] row ranges of A, or NULL: one group [0, rows)
+    int rows;                // rows when offsets == NULL
+    void* out;               // output [*, ldo]
+    int64_t ldo;             // output row stride in elements
+    const float* bias;       // EPI_F32: per-column bias or NULL
+    int32_t* status;         // device status words (MOE_ST_PIPE_TIMEOUT) or NULL
+};
+
+cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st);
+
+// device facts
+int num_sms();
+bool device_is_sm100();
+
+}  // namespace moe

@@ -1,0 +1,206 @@
+// Routing kernel: scores, selection and weights of each token, one warp per token.
+//
+// Follows the routing contract of "DSV4 Flash MoE Train-Inference Consistency Roadmap"
+// (Problem 1: logits -> top-k ids and weights with a fixed tie rule and expert bias) and
+// SpecForge PR #1003 (the selection bias moves the picks, the weights come from the
+// unbiased scores; norm_topk_prob renormalisation; route_scale for the DeepSeek seam).
+//
+// FP32 contract, bit-exact by construction: every add, multiply and divide is an
+// explicit round-to-nearest intrinsic (no contraction); the exponential is exp_rl;
+// the softmax denominator is the 32-lane tree (lane L sums experts L, L+32, ... in
+// increasing order, then butterfly levels 16, 8, 4, 2, 1); the selection compares
+// 64-bit keys (ordered choice bits, then inverted id), so ties go to the lower id.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+// exp_rl: Cody & Waite additive range reduction (x = n ln2 + r, ln2 split in a 12-bit
+// head whose products with n are exact and an fp32 tail), then the degree-7 Taylor
+// polynomial of e^r by Horner with fused multiply-adds, scaled by 2^n built from the
+// exponent field. Specials: NaN -> NaN, x < -87 -> +0, x > 88 -> +inf.
+__device__ __forceinline__ float exp_rl(float x)
+{
+    // ln 2 rounded to the nearest multiple of 2^-12 (12 significant bits: n * head is
+    // exact for |n| <= 127), and the fp32 rounding of the remainder.
+    const double kLn2 = 0.693147180559945309417232121458;
+    const float kHead = __double2float_rn(rint(kLn2 * 4096.0) / 4096.0);
+    const float kTail = __double2float_rn(kLn2 - (double)kHead);
+    const float kLog2e = __double2float_rn(1.442695040888963407359924681002);
+    if (isnan(x)) return x;
+    if (x < -87.0f) return 0.0f;
+    if (x > 88.0f) return __int_as_float(0x7f800000);
+    const float n = rintf(__fmul_rn(x, kLog2e));
+    float r = __fmaf_rn(-n, kHead, x);
+    r = __fmaf_rn(-n, kTail, r);
+    // Taylor coefficients 1/k!, k = 7 .. 0, each rounded once to fp32
+    float p = __double2float_rn(1.0 / 5040.0);
+    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 720.0));
+    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 120.0));
+    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 24.0));
+    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 6.0));
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const float two_n = __int_as_float((__float2int_rn(n) + 127) << 23);
+    return __fmul_rn(p, two_n);
+}
+
+// order-preserving 32-bit image of a choice: -0 == +0, NaN below every number
+__device__ __forceinline__ uint32_t order_bits(float c)
+{
+    if (isnan(c)) return 0u;
+    if (c == 0.0f) c = 0.0f;
+    const uint32_t u = __float_as_uint(c);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b)
+{
+    return a > b ? a : b;
+}
+
+// NE = experts held per lane (E <= 32 * NE)
+template <int NE>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
+                                                    int K, const float* __restrict__ sel_bias,
+                                                    const uint8_t* __restrict__ mask, int score_fn,
+                                                    int renorm, float route_scale,
+                                                    int32_t* __restrict__ ids,
+                                                    float* __restrict__ w, int32_t* status)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    int nan_tokens = 0, zero_den = 0;
+    for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
+         t += gridDim.x * warps_per_block) {
+        if (mask != nullptr && mask[t] == 0) {
+            if (lane < K) {
+                ids[(int64_t)t * K + lane] = -1;
+                w[(int64_t)t * K + lane] = 0.0f;
+            }
+            continue;
+        }
+        const float* row = logits + (int64_t)t * E;
+        float s[NE];
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            s[i] = (e < E) ? row[e] : 0.0f;
+        }
+        if (score_fn == MOE_SIGMOID) {
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                s[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_rl(-s[i])));
+        } else {
+            float m = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                if (lane + 32 * i < E && s[i] > m) m = s[i];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const float o = __shfl_xor_sync(0xffffffffu, m, off);
+                if (o > m) m = o;
+            }
+            float part = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                if (lane + 32 * i < E) {
+                    s[i] = exp_rl(__fsub_rn(s[i], m));
+                    part = __fadd_rn(part, s[i]);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
+#pragma unroll
+            for (int i = 0; i < NE; ++i) s[i] = __fdiv_rn(s[i], part);
+        }
+        // selection keys; empty slots get key 0 (below every real key)
+        unsigned long long key[NE];
+        bool any_nan = false;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) {
+                const float c = (sel_bias != nullptr) ? __fadd_rn(s[i], sel_bias[e]) : s[i];
+                any_nan |= isnan(c);
+                key[i] = ((unsigned long long)order_bits(c) << 32) |
+                         (unsigned long long)(0xffffffffu - (uint32_t)e);
+            } else {
+                key[i] = 0ull;
+            }
+        }
+        if (__any_sync(0xffffffffu, any_nan)) nan_tokens += (lane == 0);
+        // K rounds of a warp-wide arg-max over the remaining keys
+        int my_id = -1;
+        float my_s = 0.0f, den = 0.0f;
+        for (int j = 0; j < K; ++j) {
+            unsigned long long best = 0ull;
+#pragma unroll
+            for (int i = 0; i < NE; ++i) best = umax64(best, key[i]);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                best = umax64(best, __shfl_xor_sync(0xffffffffu, best, off));
+            const int e = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
+            const int owner = e & 31, slot = e >> 5;
+            float se = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                if (lane == owner && i == slot) {
+                    se = s[i];
+                    key[i] = 0ull;
+                }
+            }
+            se = __shfl_sync(0xffffffffu, se, owner);
+            den = (j == 0) ? se : __fadd_rn(den, se);
+            if (lane == j) { my_id = e; my_s = se; }
+        }
+        if (renorm && den == 0.0f) zero_den += (lane == 0);
+        if (lane < K) {
+            float wv;
+            if (renorm)
+                wv = (den == 0.0f) ? 0.0f : __fmul_rn(__fdiv_rn(my_s, den), route_scale);
+            else
+                wv = __fmul_rn(my_s, route_scale);
+            ids[(int64_t)t * K + lane] = my_id;
+            w[(int64_t)t * K + lane] = wv;
+        }
+    }
+    if (lane == 0) {
+        status_add(status, MOE_ST_NAN_TOKENS, nan_tokens);
+        status_add(status, MOE_ST_ZERO_DENOM, zero_den);
+    }
+}
+
+template <int NE>
+cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bias,
+                      const uint8_t* mask, int32_t* ids, float* w, int32_t* status,
+                      cudaStream_t st)
+{
+    const int threads = 256, wpb = threads / 32;
+    int blocks = (c.T + wpb - 1) / wpb;
+    const int cap = num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    route_kernel<NE><<<blocks, threads, 0, st>>>(logits, c.T, c.E, c.K, sel_bias, mask,
+                                                 c.score_fn, c.renorm, c.route_scale, ids, w,
+                                                 status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route(const moe_cfg& c, const float* logits, const float* sel_bias,
+                         const uint8_t* mask, int32_t* ids, float* w, int32_t* status,
+                         cudaStream_t st)
+{
+    const int ne = (c.E + 31) / 32;
+    if (ne <= 1) return launch_ne<1>(c, logits, sel_bias, mask, ids, w, status, st);
+    if (ne <= 2) return launch_ne<2>(c, logits, sel_bias, mask, ids, w, status, st);
+    if (ne <= 4) return launch_ne<4>(c, logits, sel_bias, mask, ids, w, status, st);
+    if (ne <= 8) return launch_ne<8>(c, logits, sel_bias, mask, ids, w, status, st);
+    if (ne <= 16) return launch_ne<16>(c, logits, sel_bias, mask, ids, w, status, st);
+    return launch_ne<32>(c, logits, sel_bias, mask, ids, w, status, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,286 @@
+"""Python binding of libmoe_b200: torch tensors in, the C ABI's calls out.
+
+Argument marshalling only -- shapes, dtypes and devices are checked, buffers are
+allocated with torch (device memory is torch's), and every step of the layer runs in
+the library's CUDA kernels on torch's current stream. Calls fail closed: a nonzero
+return code raises ``MoeError``; with ``check=True`` the stream is synchronised and a
+nonzero device status word (NaN scores, zero renormalisation denominator, bad expert
+id, pipeline timeout) raises ``StatusError`` ("DSV4 Flash MoE Train-Inference
+Consistency Roadmap", Follow-Up Issue Buckets: mismatches fail closed; UniRL PR #430:
+abort rather than continue on a parity failure).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional, Sequence
+
+import torch
+
+from . import _native as N
+
+SOFTMAX = N.MOE_SOFTMAX
+SIGMOID = N.MOE_SIGMOID
+STATUS_NAMES = ("nan_tokens", "zero_denominator", "bad_expert_id", "pipeline_timeout")
+
+
+class MoeError(RuntimeError):
+    pass
+
+
+class StatusError(MoeError):
+    def __init__(self, words):
+        self.words = list(words)
+        named = {n: w for n, w in zip(STATUS_NAMES, self.words) if w}
+        super().__init__(f"device status reports anomalies: {named}")
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    T: int
+    H: int
+    E: int
+    K: int
+    I: int
+    I_shared: int = 0
+    score_fn: int = SOFTMAX
+    renorm: bool = True
+    route_scale: float = 1.0
+
+    @classmethod
+    def of(cls, shape, T: Optional[int] = None) -> "Config":
+        """From a workload shape (anything with the same field names)."""
+        return cls(T=shape.T if T is None else T, H=shape.H, E=shape.E, K=shape.K, I=shape.I,
+                   I_shared=shape.I_shared, score_fn=shape.score_fn, renorm=bool(shape.renorm),
+                   route_scale=float(shape.route_scale))
+
+    def with_T(self, T: int) -> "Config":
+        return dataclasses.replace(self, T=T)
+
+    def c(self) -> N.MoeCfg:
+        return N.MoeCfg(self.T, self.H, self.E, self.K, self.I, self.I_shared, self.score_fn,
+                        int(bool(self.renorm)), float(self.route_scale))
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t, name, dtype, shape, dev):
+    if t is None:
+        raise MoeError(f"{name} is required")
+    if t.dtype != dtype:
+        raise MoeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise MoeError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != dev:
+        raise MoeError(f"{name}: on {t.device}, expected {dev}")
+    if not t.is_contiguous():
+        raise MoeError(f"{name} must be contiguous")
+    return t
+
+
+def _opt(t, name, dtype, shape, dev):
+    return None if t is None else _need(t, name, dtype, shape, dev)
+
+
+def _rc(code: int, what: str):
+    if code != N.MOE_OK:
+        raise MoeError(f"{what}: {N.status_string(code)} ({code})")
+
+
+def workspace_bytes(cfg: Config, stage: int) -> int:
+    return int(N.load().moe_workspace_bytes(ctypes.byref(cfg.c()), stage))
+
+
+def new_status(dev) -> torch.Tensor:
+    return torch.zeros(N.MOE_STATUS_WORDS, dtype=torch.int32, device=dev)
+
+
+def check_status(status: torch.Tensor, stream_sync: bool = True):
+    if stream_sync:
+        torch.cuda.current_stream(status.device).synchronize()
+    words = status.cpu().tolist()
+    if any(words):
+        raise StatusError(words)
+
+
+def _ws(nbytes: int, dev, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise MoeError(f"workspace of {ws.numel() * ws.element_size()} bytes < {nbytes}")
+        return ws
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+
+
+# ------------------------------------------------------------------ stages
+
+def route(cfg: Config, x=None, w_router=None, logits=None, logit_bias=None, sel_bias=None,
+          token_mask=None, status=None, check: bool = True):
+    """Routing boundary. With x: logits are computed (returned); with x=None the given
+    fp32 logits [T,E] are routed. Returns (logits, topk_ids, topk_w)."""
+    dev = (x if x is not None else logits).device
+    T, H, E, K = cfg.T, cfg.H, cfg.E, cfg.K
+    if x is not None:
+        _need(x, "x", torch.bfloat16, (T, H), dev)
+        _need(w_router, "w_router", torch.bfloat16, (E, H), dev)
+        logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits is None else logits
+    _need(logits, "logits", torch.float32, (T, E), dev)
+    _opt(logit_bias, "logit_bias", torch.float32, (E,), dev)
+    _opt(sel_bias, "sel_bias", torch.float32, (E,), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    ids = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_route(ctypes.byref(cfg.c()), _p(x), _p(w_router), _p(logit_bias),
+                           _p(sel_bias), _p(token_mask), _p(logits), _p(ids), _p(w), _p(st),
+                           _stream(dev)), "moe_route")
+    if check:
+        check_status(st)
+    return logits, ids, w
+
+
+def permute(cfg: Config, topk_ids, x=None, want_x_perm: bool = True, status=None,
+            check: bool = True):
+    """Dispatch boundary. Returns (offsets [E+1], perm_token [T*K], dest_row [T,K],
+    x_perm [T*K,H] or None)."""
+    dev = topk_ids.device
+    T, K, E, H = cfg.T, cfg.K, cfg.E, cfg.H
+    _need(topk_ids, "topk_ids", torch.int32, (T, K), dev)
+    _opt(x, "x", torch.bfloat16, (T, H), dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm_token = torch.full((T * K,), -1, dtype=torch.int32, device=dev)
+    dest_row = torch.empty(T, K, dtype=torch.int32, device=dev)
+    x_perm = None
+    if want_x_perm and x is not None:
+        x_perm = torch.empty(T * K, H, dtype=torch.bfloat16, device=dev)
+    nbytes = workspace_bytes(cfg, N.MOE_STAGE_PERMUTE)
+    ws = _ws(nbytes, dev, None)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_permute(ctypes.byref(cfg.c()), _p(topk_ids), _p(x), _p(offsets),
+                             _p(perm_token), _p(dest_row), _p(x_perm), _p(st), _p(ws),
+                             ws.numel(), _stream(dev)), "moe_permute")
+    if check:
+        check_status(st)
+    return offsets, perm_token, dest_row, x_perm
+
+
+def grouped_ffn(cfg: Config, x, x_perm, perm_token, offsets, w13, w2, w13_s=None, w2_s=None,
+                status=None, check: bool = True):
+    """Expert boundary. Returns (y [T*K,H], y_shared [T,H] or None)."""
+    dev = offsets.device
+    T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
+    _opt(x, "x", torch.bfloat16, (T, H), dev)
+    _opt(x_perm, "x_perm", torch.bfloat16, (T * K, H), dev)
+    _opt(perm_token, "perm_token", torch.int32, (T * K,), dev)
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H), dev)
+    _need(w2, "w2", torch.bfloat16, (E, H, I), dev)
+    if Is:
+        _need(w13_s, "w13_s", torch.bfloat16, (2 * Is, H), dev)
+        _need(w2_s, "w2_s", torch.bfloat16, (H, Is), dev)
+    y = torch.empty(T * K, H, dtype=torch.bfloat16, device=dev)
+    y_s = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if Is else None
+    ws = _ws(workspace_bytes(cfg, N.MOE_STAGE_FFN), dev, None)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_grouped_ffn(ctypes.byref(cfg.c()), _p(x), _p(x_perm), _p(perm_token),
+                                 _p(offsets), _p(w13), _p(w2), _p(w13_s), _p(w2_s), _p(y),
+                                 _p(y_s), _p(st), _p(ws), ws.numel(), _stream(dev)),
+        "moe_grouped_ffn")
+    if check:
+        check_status(st)
+    return y, y_s
+
+
+def combine(cfg: Config, y, topk_w, dest_row, y_shared=None, token_mask=None):
+    """Reduction boundary. Returns out [T,H] bf16."""
+    dev = y.device
+    T, H, K = cfg.T, cfg.H, cfg.K
+    if y.dim() != 2 or y.shape[1] != H or y.dtype != torch.bfloat16 or not y.is_contiguous():
+        raise MoeError("y must be a contiguous bf16 [rows, H] tensor")
+    _need(topk_w, "topk_w", torch.float32, (T, K), dev)
+    _need(dest_row, "dest_row", torch.int32, (T, K), dev)
+    _opt(y_shared, "y_shared", torch.bfloat16, (T, H), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    _rc(N.load().moe_combine(ctypes.byref(cfg.c()), _p(y), _p(topk_w), _p(dest_row),
+                             _p(y_shared), _p(token_mask), _p(out), _stream(dev)), "moe_combine")
+    return out
+
+
+# ------------------------------------------------------------------ whole layer
+
+def forward(cfg: Config, x, w_router, w13, w2, logit_bias=None, sel_bias=None, token_mask=None,
+            w13_s=None, w2_s=None, out=None, ws=None, status=None, keep: bool = False,
+            stage_events: Optional[Sequence] = None, check: bool = True):
+    """The MoE layer (routing -> dispatch -> experts -> combine) in one C-ABI call.
+
+    keep=True also returns the boundary tensors {logits, topk_ids, topk_w, offsets}.
+    stage_events: MOE_NUM_STAGE_EVENTS torch.cuda.Event(enable_timing=True) recorded at
+    the stage boundaries (for timing)."""
+    dev = x.device
+    T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
+    _need(x, "x", torch.bfloat16, (T, H), dev)
+    _need(w_router, "w_router", torch.bfloat16, (E, H), dev)
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H), dev)
+    _need(w2, "w2", torch.bfloat16, (E, H, I), dev)
+    _opt(logit_bias, "logit_bias", torch.float32, (E,), dev)
+    _opt(sel_bias, "sel_bias", torch.float32, (E,), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    if Is:
+        _need(w13_s, "w13_s", torch.bfloat16, (2 * Is, H), dev)
+        _need(w2_s, "w2_s", torch.bfloat16, (H, Is), dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, "out", torch.bfloat16, (T, H), dev)
+    ws = _ws(workspace_bytes(cfg, N.MOE_STAGE_FORWARD), dev, ws)
+    st = new_status(dev) if status is None else status
+    b = {}
+    if keep:
+        b = {"logits": torch.empty(T, E, dtype=torch.float32, device=dev),
+             "topk_ids": torch.empty(T, K, dtype=torch.int32, device=dev),
+             "topk_w": torch.empty(T, K, dtype=torch.float32, device=dev),
+             "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev)}
+    ev = None
+    if stage_events is not None:
+        if len(stage_events) != N.MOE_NUM_STAGE_EVENTS:
+            raise MoeError(f"stage_events needs {N.MOE_NUM_STAGE_EVENTS} events")
+        ev = (ctypes.c_void_p * N.MOE_NUM_STAGE_EVENTS)(
+            *[None if e is None else e.cuda_event for e in stage_events])
+    _rc(N.load().moe_forward(ctypes.byref(cfg.c()), _p(x), _p(w_router), _p(logit_bias),
+                             _p(sel_bias), _p(token_mask), _p(w13), _p(w2), _p(w13_s),
+                             _p(w2_s), _p(out), _p(b.get("logits")), _p(b.get("topk_ids")),
+                             _p(b.get("topk_w")), _p(b.get("offsets")), _p(st), _p(ws),
+                             ws.numel(), ev, _stream(dev)), "moe_forward")
+    if check:
+        check_status(st)
+    return (out, b) if keep else out
+
+
+class MoELayer:
+    """A layer holding its weights and a reusable workspace sized for up to max_T tokens.
+
+    weights: dict with w_router, w13, w2 and optionally logit_bias, sel_bias, w13_s, w2_s
+    (the layout of include/moe.h)."""
+
+    def __init__(self, cfg: Config, weights: dict, max_T: Optional[int] = None):
+        self.cfg = cfg
+        self.w = weights
+        self.max_T = cfg.T if max_T is None else max_T
+        dev = weights["w13"].device
+        self.ws = _ws(workspace_bytes(cfg.with_T(self.max_T), N.MOE_STAGE_FORWARD), dev, None)
+        self.status = new_status(dev)
+
+    def __call__(self, x, token_mask=None, out=None, keep=False, check=True, stage_events=None):
+        T = x.shape[0]
+        if T > self.max_T:
+            raise MoeError(f"{T} tokens > the layer's max_T {self.max_T}")
+        w = self.w
+        return forward(self.cfg.with_T(T), x, w["w_router"], w["w13"], w["w2"],
+                       logit_bias=w.get("logit_bias"), sel_bias=w.get("sel_bias"),
+                       token_mask=token_mask, w13_s=w.get("w13_s"), w2_s=w.get("w2_s"),
+                       out=out, ws=self.ws, status=self.status, keep=keep, check=check,
+                       stage_events=stage_events)

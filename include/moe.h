@@ -1,0 +1,230 @@
+/*
+ * moe.h -- C ABI of libmoe_b200: the forward pass of a top-k mixture-of-experts FFN
+ * layer with a bitwise consistency contract, as hand-written sm_100a (B200) kernels.
+ *
+ * The layer (the semantic boundaries named in "DSV4 Flash MoE Train-Inference
+ * Consistency Roadmap", Problem 2, and the MoE layer of SpecForge PR #1003):
+ *
+ *   logits = x . W_router^T (+ logit_bias)                     routing boundary
+ *   s      = softmax(logits) or sigmoid(logits)               (unbiased scores)
+ *   ids    = top-k of s + sel_bias, ties -> lower expert id
+ *   w      = s[ids] / sum(s[ids]) * route_scale   (renorm)   or s[ids] * route_scale
+ *   rows   = stable counting sort of the (token, rank) pairs by expert      dispatch
+ *   y_r    = W2_e . (silu(W1g_e . x_t) * (W1u_e . x_t))  per dispatched row   experts
+ *   out_t  = bf16( sum_j w_j * y_{row(t,j)}  [+ y_shared_t] )  fixed order   reduction
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers of the current CUDA device, row-major,
+ *    densely packed, 16-byte aligned. bf16 tensors are passed as uint16_t* (raw bits).
+ *  - The caller owns every buffer, including the workspace. The library allocates no
+ *    device memory and keeps no per-call state; it caches only immutable per-device
+ *    facts (SM count, kernel attributes, the driver's tensor-map encoder).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only enqueue work
+ *    on it and never synchronise the host, so they can be captured in a CUDA graph.
+ *  - Return value: MOE_OK (0) or a negative MOE_ERR_* code. Arguments are validated on
+ *    the host before anything is enqueued; on an error nothing is enqueued.
+ *  - Data anomalies found on the device (NaN scores, a zero renormalisation
+ *    denominator, expert ids out of range, a tensor-core pipeline wait that gave up)
+ *    are counted in `status`, an int32[MOE_STATUS_WORDS] device array that the entry
+ *    point clears at its start. Nothing traps or asserts on the device. Callers that
+ *    want the fail-closed behaviour of the contract read `status` after the stream
+ *    and reject the result when a word is nonzero (the Python binding does).
+ *  - Results are bitwise reproducible: for a given build and GPU, a token's routes and
+ *    output depend only on its own row and the weights -- never on T, on padding, on
+ *    the order of the other tokens or on how a batch is split into calls.
+ *
+ * Shapes supported: 1 <= E <= 1024, 1 <= K <= min(E, 16), H % 128 == 0 and
+ * 128 <= H <= 16384, I % 128 == 0, I_shared % 128 == 0 (0 = no shared expert),
+ * 0 <= T and T * K < 2^31. T == 0 is a no-op.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define MOE_API __declspec(dllexport)
+#else
+#define MOE_API __attribute__((visibility("default")))
+#endif
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_ARG (-1)           /* a required pointer is NULL or misaligned */
+#define MOE_ERR_SHAPE (-2)         /* a size outside the supported shapes */
+#define MOE_ERR_WORKSPACE (-3)     /* ws_bytes smaller than moe_workspace_bytes() */
+#define MOE_ERR_CUDA (-4)          /* a CUDA runtime/driver call or a launch failed */
+#define MOE_ERR_UNIMPLEMENTED (-5) /* a valid request this build does not serve */
+#define MOE_ERR_DEVICE (-6)        /* the current device is not sm_100 */
+
+/* score functions */
+#define MOE_SOFTMAX 0
+#define MOE_SIGMOID 1
+
+/* words of the device status array */
+#define MOE_ST_NAN_TOKENS 0     /* tokens with a NaN selection score */
+#define MOE_ST_ZERO_DENOM 1     /* tokens whose renormalisation denominator was 0 */
+#define MOE_ST_BAD_EXPERT_ID 2  /* expert ids >= E met by the dispatch (not counting -1) */
+#define MOE_ST_PIPE_TIMEOUT 3   /* a tensor-core pipeline wait gave up (result invalid) */
+#define MOE_STATUS_WORDS 8
+
+/* stages, for moe_workspace_bytes */
+#define MOE_STAGE_ROUTE 0
+#define MOE_STAGE_PERMUTE 1
+#define MOE_STAGE_FFN 2
+#define MOE_STAGE_COMBINE 3
+#define MOE_STAGE_FORWARD 4
+
+/* number of CUDA events moe_forward can record (stage boundaries), see moe_forward */
+#define MOE_NUM_STAGE_EVENTS 8
+
+typedef struct moe_cfg {
+    int32_t T;           /* tokens in this call */
+    int32_t H;           /* hidden size */
+    int32_t E;           /* routed experts */
+    int32_t K;           /* experts per token (top-k) */
+    int32_t I;           /* routed expert intermediate size */
+    int32_t I_shared;    /* shared (always-on) expert intermediate size, 0 = none */
+    int32_t score_fn;    /* MOE_SOFTMAX or MOE_SIGMOID */
+    int32_t renorm;      /* 1: weights renormalised over the K selected scores */
+    float route_scale;   /* weights are multiplied by it (1.0 = unchanged) */
+} moe_cfg;
+
+/*
+ * Bytes of workspace the given stage needs for cfg (MOE_STAGE_FORWARD: moe_forward).
+ * Returns 0 for an invalid cfg as well as for stages that need none.
+ */
+MOE_API size_t moe_workspace_bytes(const moe_cfg* cfg, int stage);
+
+/*
+ * Routing boundary ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 1
+ * "Routing Is A Discrete Decision": router logits, top-k ids, top-k weights and the
+ * tie rule; SpecForge PR #1003, the selection-bias commit: the bias shifts only the
+ * picks, the weights come from the unbiased scores).
+ *
+ *  x          [T,H] bf16, or NULL: then `logits` is an INPUT ([T,E] fp32) and the
+ *             router product is skipped (replaying or injecting logits).
+ *  w_router   [E,H] bf16 (ignored when x is NULL).
+ *  logit_bias [E] fp32 or NULL, added to the logits (part of the logits, not of the
+ *             selection).
+ *  sel_bias   [E] fp32 or NULL: choice = score + sel_bias selects the experts; the
+ *             weights still use the unbiased score.
+ *  token_mask [T] uint8 or NULL (all tokens real): a 0 marks padding; such tokens get
+ *             ids -1 and weights 0 and are skipped by every later stage.
+ *  logits     [T,E] fp32: output (x given) or input (x NULL).
+ *  topk_ids   [T,K] int32 out, rank order (rank 0 = best).
+ *  topk_w     [T,K] fp32 out.
+ *  status     int32[MOE_STATUS_WORDS] device, cleared then counted; may be NULL.
+ * Score arithmetic is the FP32 contract: exp_rl, the 32-lane softmax tree, IEEE
+ * round-to-nearest adds/multiplies/divides, no FMA contraction outside exp_rl.
+ */
+MOE_API int moe_route(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                      const float* logit_bias, const float* sel_bias,
+                      const uint8_t* token_mask, float* logits, int32_t* topk_ids,
+                      float* topk_w, int32_t* status, void* stream);
+
+/*
+ * Dispatch boundary ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 2:
+ * token-to-expert map and valid token counts). A stable counting sort of the T*K
+ * assignments a = t*K + j by expert id, ties kept in increasing a.
+ *
+ *  topk_ids   [T,K] int32 (-1 = not routed, e.g. padding; ids >= E are counted in
+ *             status[MOE_ST_BAD_EXPERT_ID] and not routed).
+ *  x          [T,H] bf16 or NULL; with x and x_perm given, row r of x_perm receives
+ *             x[perm_token[r]].
+ *  offsets    [E+1] int32 out: rows of expert e are offsets[e] .. offsets[e+1]-1.
+ *  perm_token [T*K] int32 out: row -> token (rows >= offsets[E] are left untouched).
+ *  dest_row   [T*K] int32 out: assignment -> row, -1 when not routed.
+ *  x_perm     [T*K,H] bf16 out or NULL.
+ *  ws         moe_workspace_bytes(cfg, MOE_STAGE_PERMUTE) bytes of device scratch.
+ */
+MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint16_t* x,
+                        int32_t* offsets, int32_t* perm_token, int32_t* dest_row,
+                        uint16_t* x_perm, int32_t* status, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * Expert boundary ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 2:
+ * gate_and_up -> down; SpecForge PR #1003, experts.py: grouped experts and the
+ * always-on shared expert). Grouped SwiGLU GEMMs on the tensor cores:
+ *   h_r = bf16( silu(x_r . W13[e, 0:I]^T) * (x_r . W13[e, I:2I]^T) )   (fp32 accumulate)
+ *   y_r = bf16( h_r . W2[e]^T )                                        (fp32 accumulate)
+ * for every row r of expert e, with a reduction order that is fixed per (H, I): never
+ * a function of T, of the rows per expert or of the row's place in a tile.
+ *
+ *  x          [T,H] bf16 tokens (read by the shared expert, and by the routed experts
+ *             through perm_token when x_perm is NULL).
+ *  x_perm     [T*K,H] bf16 dispatched rows (from moe_permute), or NULL to gather the
+ *             rows from x via perm_token inside the GEMM.
+ *  perm_token [T*K] int32 from moe_permute (required when x_perm is NULL).
+ *  offsets    [E+1] int32 from moe_permute.
+ *  w13        [E, 2I, H] bf16: rows 0..I-1 gate, rows I..2I-1 up (each row K-major).
+ *  w2         [E, H, I] bf16.
+ *  w13_s, w2_s  shared expert [2*I_shared, H] and [H, I_shared] bf16, or NULL.
+ *  y          [T*K, H] bf16 out, row r = output of dispatched row r.
+ *  y_shared   [T, H] bf16 out (required when the shared expert is given).
+ *  status     as in moe_route (only MOE_ST_PIPE_TIMEOUT is used here), may be NULL.
+ *  ws         moe_workspace_bytes(cfg, MOE_STAGE_FFN) bytes.
+ */
+MOE_API int moe_grouped_ffn(const moe_cfg* cfg, const uint16_t* x, const uint16_t* x_perm,
+                            const int32_t* perm_token, const int32_t* offsets,
+                            const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
+                            const uint16_t* w2_s, uint16_t* y, uint16_t* y_shared,
+                            int32_t* status, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Reduction boundary ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 3
+ * "Final Reduction Is The Core Drift Point"; "From Expert Reduction to Behavioral
+ * Divergence", Abstract: the order of the expert sum is part of the contract).
+ * Per token t and column h, in FP32 with IEEE round-to-nearest and no FMA:
+ *   acc = w_0 * y[dest_row[t,0], h]; acc += w_j * y[dest_row[t,j], h] for j = 1..K-1
+ *   (each product rounded, rank order, terms with dest_row < 0 skipped),
+ *   then acc += y_shared[t, h] if given; out = bf16 round-to-nearest-even(acc).
+ * Tokens with token_mask[t] == 0 get out = 0.
+ *
+ *  y [T*K,H] bf16, topk_w [T,K] fp32, dest_row [T,K] int32, y_shared [T,H] bf16 or NULL,
+ *  token_mask [T] uint8 or NULL, out [T,H] bf16.
+ */
+MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* y, const float* topk_w,
+                        const int32_t* dest_row, const uint16_t* y_shared,
+                        const uint8_t* token_mask, uint16_t* out, void* stream);
+
+/*
+ * The whole layer (SpecForge PR #1003, layer.py: MoELayer = router + routed experts +
+ * optional shared expert): moe_route -> moe_permute -> moe_grouped_ffn -> moe_combine
+ * on one stream, intermediates in `ws`.
+ *
+ *  Inputs as in the stages above; out [T,H] bf16.
+ *  Optional boundary outputs (NULL = not kept): logits [T,E] fp32, topk_ids [T,K],
+ *  topk_w [T,K], offsets [E+1].
+ *  status     int32[MOE_STATUS_WORDS] device, required.
+ *  ws         moe_workspace_bytes(cfg, MOE_STAGE_FORWARD) bytes.
+ *  stage_events NULL, or MOE_NUM_STAGE_EVENTS cudaEvent_t handles recorded on `stream`
+ *             at the stage boundaries: [0] start, [1] after router logits, [2] after
+ *             routing, [3] after dispatch, [4] after gate_up, [5] after down, [6] after
+ *             the shared expert, [7] after the combine (timing only).
+ */
+MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                        const float* logit_bias, const float* sel_bias,
+                        const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                        const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out,
+                        float* logits, int32_t* topk_ids, float* topk_w, int32_t* offsets,
+                        int32_t* status, void* ws, size_t ws_bytes, void* const* stage_events,
+                        void* stream);
+
+/* Text of a return code. */
+MOE_API const char* moe_status_string(int code);
+
+/* ABI version of this header (major * 100 + minor). */
+MOE_API int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,115 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol include/moe.h
+declares, and rejects bad arguments on the host before touching the device (no GPU is
+needed and no CUDA call is reached)."""
+import ctypes
+import re
+
+import pytest
+
+from deterministic_invariant_routing_b200 import _native as N
+from deterministic_invariant_routing_b200 import build, moe
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return N.load()
+
+
+def declared_symbols():
+    with open(N.HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    raw = ctypes.CDLL(N.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(N.SIGNATURES)
+
+
+def test_header_constants_match_binding():
+    with open(N.HEADER_PATH) as f:
+        text = f.read()
+    for name, val in re.findall(r"#define\s+(MOE_\w+)\s+\(?(-?\d+)\)?", text):
+        assert getattr(N, name) == int(val), name
+
+
+def test_status_strings(lib):
+    assert N.status_string(0) == "ok"
+    for code in (-1, -2, -3, -4, -5, -6):
+        assert N.status_string(code) != "unknown status"
+    assert lib.moe_abi_version() == 100
+
+
+GOOD = dict(T=64, H=128, E=8, K=2, I=256)
+
+
+def cfg(**over):
+    d = dict(GOOD)
+    d.update(over)
+    return moe.Config(**d).c()
+
+
+@pytest.mark.parametrize("over", [dict(H=100), dict(H=64), dict(I=100), dict(E=0),
+                                  dict(E=1025), dict(K=0), dict(K=17), dict(K=9, E=8),
+                                  dict(I_shared=100), dict(T=-1), dict(score_fn=2),
+                                  dict(T=200_000_000, K=16)])
+def test_bad_shapes_rejected(lib, over):
+    c = cfg(**over)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    assert lib.moe_route(ctypes.byref(c), fake, fake, None, None, None, fake, fake, fake, None,
+                         None) == N.MOE_ERR_SHAPE
+    assert lib.moe_workspace_bytes(ctypes.byref(c), N.MOE_STAGE_FORWARD) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    c = cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.moe_route(ctypes.byref(c), fake, None, None, None, None, fake, fake, fake, None,
+                         None) == N.MOE_ERR_ARG
+    assert lib.moe_route(ctypes.byref(c), odd, fake, None, None, None, fake, fake, fake, None,
+                         None) == N.MOE_ERR_ARG
+    assert lib.moe_combine(ctypes.byref(c), None, fake, fake, None, None, fake, None) == N.MOE_ERR_ARG
+    assert lib.moe_combine(ctypes.byref(c), odd, fake, fake, None, None, fake, None) == N.MOE_ERR_ARG
+    args = [fake] * 10
+    assert lib.moe_forward(None, *args, fake, fake, fake, fake, fake, fake, 1 << 40, None,
+                           None) == N.MOE_ERR_ARG
+
+
+def test_workspace_checks(lib):
+    c = cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    need = lib.moe_workspace_bytes(ctypes.byref(c), N.MOE_STAGE_FORWARD)
+    assert need > 64 * 2 * 128 * 2  # at least x_perm
+    rc = lib.moe_forward(ctypes.byref(c), fake, fake, None, None, None, fake, fake, None, None,
+                         fake, None, None, None, None, fake, fake, need - 1, None, None)
+    assert rc == N.MOE_ERR_WORKSPACE
+    rc = lib.moe_permute(ctypes.byref(c), fake, None, fake, fake, fake, None, None, fake, 0, None)
+    assert rc == N.MOE_ERR_WORKSPACE
+    # T == 0 is a no-op that succeeds without touching the device
+    c0 = cfg(T=0)
+    need0 = lib.moe_workspace_bytes(ctypes.byref(c0), N.MOE_STAGE_FORWARD)
+    rc = lib.moe_forward(ctypes.byref(c0), fake, fake, None, None, None, fake, fake, None, None,
+                         fake, None, None, None, None, fake, fake, need0, None, None)
+    assert rc == N.MOE_OK
+
+
+def test_workspace_sizes_scale_with_tokens(lib):
+    a = lib.moe_workspace_bytes(ctypes.byref(cfg(T=1000)), N.MOE_STAGE_FORWARD)
+    b = lib.moe_workspace_bytes(ctypes.byref(cfg(T=2000)), N.MOE_STAGE_FORWARD)
+    assert 1.8 < b / a < 2.2
+    s = lib.moe_workspace_bytes(ctypes.byref(cfg(I_shared=512)), N.MOE_STAGE_FFN)
+    n = lib.moe_workspace_bytes(ctypes.byref(cfg()), N.MOE_STAGE_FFN)
+    assert s > n
+
+
+def test_binding_refuses_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(N, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(N, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        N.load()

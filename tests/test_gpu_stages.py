@@ -1,0 +1,157 @@
+"""Level-1 parity of the integer and FP32-contract stages: the CUDA route, dispatch and
+combine kernels against the oracle, bit for bit, on the same inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from deterministic_invariant_routing_b200 import moe, synthetic
+from deterministic_invariant_routing_b200 import _native as N
+from helpers import DEV, bits
+
+pytestmark = pytest.mark.gpu
+
+SM, SG = moe.SOFTMAX, moe.SIGMOID
+
+
+def adversarial_logits(T, E, seed, std=3.0):
+    """Random logits with injected exact ties (at every rank), all-equal rows, signed
+    zeros, -inf, a NaN row and a wide dynamic range (exp_rl's full input domain)."""
+    l = synthetic.random_logits(T, E, seed, std=std).numpy()
+    rng = np.random.default_rng(seed)
+    for t in range(0, min(T, 40)):
+        i, j = rng.choice(E, 2, replace=False) if E > 1 else (0, 0)
+        l[t, j] = l[t, i]
+    if T > 45:
+        l[41] = 0.5
+        l[42, :] = -0.0
+        l[42, ::2] = 0.0
+        l[43, : max(1, E // 2)] = -np.inf
+        l[44] = rng.uniform(-80, 80, E)
+        l[45, rng.integers(0, E)] = np.nan
+    return np.ascontiguousarray(l.astype(np.float32))
+
+
+ROUTE_CASES = [
+    # E, K, score_fn, renorm, route_scale, with_bias, T
+    (8, 2, SM, 1, 1.0, False, 64),
+    (8, 1, SM, 0, 1.0, True, 1000),
+    (128, 8, SM, 1, 1.0, False, 3001),
+    (256, 6, SG, 1, 2.5, True, 2048),
+    (1024, 16, SM, 1, 1.0, True, 517),
+    (33, 3, SG, 0, 1.0, False, 700),
+    (1, 1, SM, 1, 1.0, False, 50),
+    (100, 7, SM, 1, 0.5, True, 999),
+]
+
+
+@pytest.mark.parametrize("E,K,score_fn,renorm,scale,with_bias,T", ROUTE_CASES)
+def test_route_bit_exact(E, K, score_fn, renorm, scale, with_bias, T):
+    seed = 100 + E + K
+    l = adversarial_logits(T, E, seed)
+    bias = synthetic.uniform_f32(E, 0.05, seed, "sel_bias").numpy() if with_bias else None
+    mask = synthetic.random_mask(T, 0.9, seed).numpy()
+    cfg = moe.Config(T=T, H=128, E=E, K=K, I=128, score_fn=score_fn, renorm=bool(renorm),
+                     route_scale=scale)
+    st = moe.new_status(DEV)
+    _, ids, w = moe.route(cfg, logits=torch.from_numpy(l).to(DEV),
+                          sel_bias=None if bias is None else torch.from_numpy(bias).to(DEV),
+                          token_mask=torch.from_numpy(mask).to(DEV), status=st, check=False)
+    torch.cuda.synchronize()
+    r_ids, r_w, r_st = oracle.route_fp32(l, K, score_fn, renorm, scale, sel_bias=bias, mask=mask)
+    g_ids = ids.cpu().numpy()
+    g_w = w.cpu().numpy()
+    assert np.array_equal(g_ids, r_ids), np.argwhere(g_ids != r_ids)[:5]
+    nan = np.isnan(r_w)
+    assert np.array_equal(np.isnan(g_w), nan)
+    assert np.array_equal(g_w[~nan].view(np.uint32), r_w[~nan].view(np.uint32))
+    s = st.cpu().numpy()
+    assert s[N.MOE_ST_NAN_TOKENS] == r_st[0] and s[N.MOE_ST_ZERO_DENOM] == r_st[1]
+
+
+def test_route_golden_two_token(golden):
+    g = golden("two_token_route_combine.json")
+    l = np.array(g["logits"], np.float32)
+    cfg = moe.Config(T=2, H=128, E=g["E"], K=g["K"], I=128, renorm=True)
+    _, ids, w = moe.route(cfg, logits=torch.from_numpy(l).to(DEV),
+                          sel_bias=torch.tensor(g["sel_bias"], dtype=torch.float32, device=DEV))
+    assert ids.cpu().tolist() == g["expect_ids"]
+    assert w.cpu().tolist() == g["expect_w"]
+    offsets, perm_token, dest_row, _ = moe.permute(cfg, ids)
+    assert offsets.cpu().tolist() == g["expect_offsets"]
+    assert dest_row.cpu().tolist() == g["expect_dest_row"]
+    assert perm_token.cpu().tolist()[:4] == g["expect_perm_token"]
+    # combine on 128 columns: the fixture's 4 columns, zeros after them
+    y = torch.zeros(4, 128, dtype=torch.bfloat16)
+    y[:, :4] = torch.tensor(g["y"])
+    ys = torch.zeros(2, 128, dtype=torch.bfloat16)
+    ys[:, :4] = torch.tensor(g["y_shared"])
+    out = moe.combine(cfg, y.to(DEV), w, dest_row, y_shared=ys.to(DEV))
+    ob = bits(out)
+    assert [[f"{v:04x}" for v in row[:4]] for row in ob] == g["expect_out_bf16_hex"]
+    assert np.all(ob[:, 4:] == 0)
+
+
+@pytest.mark.parametrize("T,K,E", [(1, 1, 8), (64, 2, 8), (3001, 8, 128), (8192, 1, 8),
+                                   (2048, 6, 256), (777, 16, 1024), (20000, 8, 128)])
+def test_permute_bit_exact(T, K, E):
+    rng = np.random.default_rng(T + K + E)
+    # skewed expert choice (uneven loads, some experts empty), masked tokens, bad ids
+    p = rng.dirichlet(np.full(E, 0.3))
+    ids = np.stack([rng.choice(E, K, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    ids[rng.random(T) < 0.1] = -1
+    n_bad = 0
+    if T > 10:
+        ids[5, 0] = E + 3
+        n_bad = 1
+    H = 256
+    x = synthetic.normal_bf16(T, H, 1.0, 7, "x")
+    cfg = moe.Config(T=T, H=H, E=E, K=K, I=128)
+    st = moe.new_status(DEV)
+    offsets, perm_token, dest_row, x_perm = moe.permute(
+        cfg, torch.from_numpy(ids).to(DEV), x=x.to(DEV), status=st, check=False)
+    r_off, r_perm, r_dest, r_bad = oracle.permute(ids, E)
+    assert np.array_equal(offsets.cpu().numpy(), r_off)
+    n = int(r_off[-1])
+    assert np.array_equal(perm_token.cpu().numpy()[:n], r_perm[:n])
+    assert np.array_equal(dest_row.cpu().numpy(), r_dest)
+    assert np.array_equal(bits(x_perm[:n]), bits(x)[r_perm[:n]])
+    assert st.cpu().numpy()[N.MOE_ST_BAD_EXPERT_ID] == r_bad == n_bad
+
+
+@pytest.mark.parametrize("T,K,H,shared,masked", [(1, 1, 128, False, False),
+                                                  (64, 2, 128, False, True),
+                                                  (1000, 8, 2048, False, True),
+                                                  (333, 6, 4096, True, True),
+                                                  (4096, 1, 4096, False, False),
+                                                  (100, 16, 256, True, False)])
+def test_combine_bit_exact(T, K, H, shared, masked):
+    rng = np.random.default_rng(T * 7 + K)
+    rows = T * K
+    y = synthetic.normal_bf16(rows, H, 1.5, T + K, "x")
+    ys = synthetic.normal_bf16(T, H, 1.0, T + K, "fill") if shared else None
+    w = rng.uniform(0, 1, (T, K)).astype(np.float32)
+    dest = rng.permutation(rows).astype(np.int32).reshape(T, K)
+    mask = (rng.random(T) > 0.2).astype(np.uint8) if masked else None
+    if masked:
+        dest[mask == 0] = -1
+    if T > 3 and K > 1:
+        dest[3, K - 1] = -1  # a skipped term inside a live token
+    cfg = moe.Config(T=T, H=H, E=max(K, 8), K=K, I=128)
+    out = moe.combine(cfg, y.to(DEV), torch.from_numpy(w).to(DEV), torch.from_numpy(dest).to(DEV),
+                      y_shared=None if ys is None else ys.to(DEV),
+                      token_mask=None if mask is None else torch.from_numpy(mask).to(DEV))
+    ref = oracle.combine_fp32(y, w, dest, ys, mask)
+    assert np.array_equal(bits(out), ref)
+
+
+def test_combine_cancellation_order(golden):
+    c = golden("tree_sum_and_combine_order.json")["combine_case"]
+    K, H = c["K"], 128
+    y = torch.zeros(K, H, dtype=torch.bfloat16)
+    y[:, 0] = torch.tensor([r[0] for r in c["y"]])
+    w = torch.tensor(c["w"], dtype=torch.float32)
+    d = torch.tensor(c["dest_row"], dtype=torch.int32)
+    cfg = moe.Config(T=1, H=H, E=8, K=K, I=128)
+    out = moe.combine(cfg, y.to(DEV), w.to(DEV), d.to(DEV))
+    assert out.float().cpu()[0, 0].item() == c["expect_acc"][0][0]
