@@ -1,0 +1,335 @@
+#!/usr/bin/env python
+"""MoE-layer throughput on B200: tokens/s of the batch-invariant top-k MoE FFN forward
+(bf16, fp32 accumulate) and its fraction of the tensor/HBM roofline.
+
+One step = one moe_forward over a batch of synthetic tokens already resident in HBM:
+router logits -> routing -> dispatch -> grouped gate_up/SwiGLU -> grouped down ->
+(shared expert) -> fixed-order combine. Default workload: the Qwen3-30B-A3B-shaped layer
+(hidden 2048, 128 experts x 768, top-8 softmax, renormalised) at T = 16384 tokens.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch one process per GPU with torch.distributed.run; every rank runs an
+independent replica of the layer on its own tokens (the layer has no cross-token
+exchange), the time is the max over ranks, and value = all ranks' tokens / that time.
+`--impl reference` times the plain CPU oracle (the correctness reference, run as it
+stands on the host cores) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CPU_SAMPLE_SECONDS = 15.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="qwen3_30b_a3b")
+    p.add_argument("--T", type=int, default=16384)
+    p.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch of a kernel from a committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+        if rec["source_sha"] != source_sha(rec["source"]):
+            return None
+        return rec["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": mx or None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def layer_work(s, n_touched):
+    """Algorithmic FLOPs and bytes of one layer forward (intermediates excluded)."""
+    T, H, E, K, I, Is = s.T, s.H, s.E, s.K, s.I, s.I_shared
+    flops = T * K * (4 * H * I + 2 * I * H) + T * 6 * H * Is + 2 * T * H * E
+    byts = (n_touched * 3 * H * I * 2 + 3 * H * Is * 2 + 2 * T * H * 2 + E * H * 2
+            + T * K * 8)
+    return flops, byts
+
+
+def _calibrate(s, d_cpu):
+    """Seconds per token of the oracle's layer forward with every host core busy."""
+    import numpy as np
+
+    import oracle
+    n = max(oracle.num_threads(), 2)
+    sel = np.arange(min(n, s.T), dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.layer_forward(s, d_cpu, sel)
+    return max((time.perf_counter() - t0) / sel.size, 1e-6)
+
+
+def cpu_baseline(s, d_cpu, seconds=CPU_SAMPLE_SECONDS, per_tok=None, seed=0):
+    """The oracle's whole-layer forward on a bounded token sample, tokens/s."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(seed)
+    if per_tok is None:
+        per_tok = _calibrate(s, d_cpu)
+    n = int(min(max(seconds / per_tok, 1), s.T))
+    sel = np.sort(rng.choice(s.T, n, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.layer_forward(s, d_cpu, sel)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of the {s.T} tokens of the same layer (full layer per token: FP64 "
+                      f"router, FP32-contract routing, FP64 experts), {dt:.2f} s"}
+
+
+def run_reference(a):
+    """The correctness reference (the CPU oracle, as it stands) on the host cores; each
+    step is a bounded token sample, the whole run about 90 s."""
+    from deterministic_invariant_routing_b200 import synthetic
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s, d = synthetic.make_layer(a.workload, T=a.T, device="cpu")
+    per_tok = _calibrate(s, d)
+    secs = max(90.0 / (a.warmup + a.steps), per_tok)
+    per_step = []
+    for i in range(a.warmup + a.steps):
+        r = cpu_baseline(s, d, seconds=secs, per_tok=per_tok, seed=i)
+        if i >= a.warmup:
+            per_step.append(r)
+    value = statistics.median(r["value"] for r in per_step)
+    cb = dict(per_step[-1], value=value)
+    cb["sample"] = f"per step: {per_step[-1]['sample']}"
+    line = {"impl": "reference", "metric": "MoE-layer tokens/s (bf16, batch-invariant)",
+            "value": value, "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": 1e3 * s.T / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(s, a.gpus), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(s, n):
+    return {"workload": f"{s.name}_T{s.T}", "T_per_gpu": s.T, "H": s.H, "E": s.E, "K": s.K,
+            "I": s.I, "I_shared": s.I_shared,
+            "score_fn": "sigmoid" if s.score_fn == 1 else "softmax", "renorm": bool(s.renorm),
+            "route_scale": s.route_scale, "global_tokens": s.T * n,
+            "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
+            "l2": "inputs larger than L2 (expert weights and per-step intermediates exceed "
+                  "126 MB), no flush"}
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+
+    import torch
+    import torch.distributed as dist
+
+    from deterministic_invariant_routing_b200 import moe, synthetic
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    s = synthetic.shape(a.workload, T=a.T)
+    weights = synthetic.make_weights(s, device=dev)
+    x = synthetic.make_tokens(s, s.T, seed=s.seed + 1000 * rank, device=dev)
+    cfg = moe.Config.of(s)
+    layer = moe.MoELayer(cfg, weights)
+
+    for _ in range(a.warmup):
+        layer(x, check=False)
+    out, b = layer(x, keep=True, check=True)  # fail closed once before timing
+    offsets = b["offsets"].cpu()
+    n_touched = int(((offsets[1:] - offsets[:-1]) > 0).sum())
+    rows = int(offsets[-1])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    K = a.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    barrier()
+    with ClockSampler(gpu_id) as clk:
+        start.record()
+        for k in range(K):
+            layer(x, check=False, stage_events=ev[k])
+        stop.record()
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(stop) / K)
+    moe.check_status(layer.status)
+
+    def stage_ms(i, j):
+        return statistics.fmean(e[i].elapsed_time(e[j]) for e in ev)
+
+    stages = {"router_gemm": stage_ms(0, 1), "route": stage_ms(1, 2), "dispatch": stage_ms(2, 3),
+              "gate_up_gemm": stage_ms(3, 4), "down_gemm": stage_ms(4, 5),
+              "shared_expert": stage_ms(5, 6), "combine": stage_ms(6, 7)}
+
+    # end to end through the public call with host buffers: H2D of x, forward, D2H of out
+    Ke = a.e2e_steps or K
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_d = torch.empty_like(x)
+    for _ in range(3):
+        x_d.copy_(x_h, non_blocking=True)
+        out_h.copy_(layer(x_d, check=False), non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(Ke):
+        x_d.copy_(x_h, non_blocking=True)
+        o = layer(x_d, check=False)
+        out_h.copy_(o, non_blocking=True)
+    e1.record()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / Ke)
+    moe.check_status(layer.status)
+
+    pk, pk_src = peaks()
+    flops, byts = layer_work(s, n_touched)
+    gate_flops = 4 * rows * s.H * s.I
+    gate_ms = max_over_ranks(stages["gate_up_gemm"])
+    achieved = gate_flops / (gate_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    t_roof = max(flops / (peak * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    clocks = clk.summary()
+    line = {
+        "metric": "MoE-layer tokens/s (bf16, batch-invariant)",
+        "value": s.T * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(s, world),
+        "roofline": {"bound": "tensor", "kernel": "gate_up grouped GEMM (tcgen05)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": ncu_traffic("gate_up"),
+                     "peak_source": f"{pk_src} bf16 sustained",
+                     "algorithmic_flops_per_launch": gate_flops},
+        "layer_roofline": {"flops": flops, "bytes": byts, "roofline_ms": t_roof * 1e3,
+                           "frac": t_roof * 1e3 / ms, "experts_touched": n_touched,
+                           "peaks": f"{pk_src}: {peak} TFLOP/s bf16 sustained, "
+                                    f"{pk['hbm_gbs']} GB/s"},
+        "stage_ms": stages,
+        "e2e": {"value": s.T * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": K * (9 + (2 if s.I_shared else 0)),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        d_cpu = {k: (None if v is None else v.cpu()) for k, v in weights.items()}
+        d_cpu["x"] = x.cpu()
+        line["cpu_baseline"] = cpu_baseline(s, d_cpu)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

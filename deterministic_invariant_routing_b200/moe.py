@@ -248,6 +248,10 @@ def forward(cfg: Config, x, w_router, w13, w2, logit_bias=None, sel_bias=None, t
     if stage_events is not None:
         if len(stage_events) != N.MOE_NUM_STAGE_EVENTS:
             raise MoeError(f"stage_events needs {N.MOE_NUM_STAGE_EVENTS} events")
+        stream = torch.cuda.current_stream(dev)
+        for e in stage_events:
+            if e is not None and not e.cuda_event:
+                e.record(stream)  # torch creates its events lazily, on first record
         ev = (ctypes.c_void_p * N.MOE_NUM_STAGE_EVENTS)(
             *[None if e is None else e.cuda_event for e in stage_events])
     _rc(N.load().moe_forward(ctypes.byref(cfg.c()), _p(x), _p(w_router), _p(logit_bias),
