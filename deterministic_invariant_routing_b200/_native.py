@@ -54,6 +54,7 @@ SIGNATURES = {
     "moe_workspace_bytes": (_SZ, [_CFG, _I]),
     "moe_route": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_permute_noalloc": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_combine": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,

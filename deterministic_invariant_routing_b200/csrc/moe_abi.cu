@@ -286,6 +286,30 @@ MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint1
     return cuda_rc(launch_gather_rows(*cfg, x, perm_token, offsets, x_perm, st));
 }
 
+MOE_API int moe_permute_noalloc(const moe_cfg* cfg, const int32_t* topk_ids, const uint16_t* x,
+                                int32_t* offsets, int32_t* perm_token, int32_t* dest_row,
+                                uint16_t* x_perm, int32_t* status, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (topk_ids == nullptr || offsets == nullptr || perm_token == nullptr || dest_row == nullptr)
+        return MOE_ERR_ARG;
+    if (x_perm != nullptr && (x == nullptr || !aligned16(x) || !aligned16(x_perm)))
+        return MOE_ERR_ARG;
+    if (permute_ws_bytes(*cfg) > (size_t)kPermuteFixedScratchInts * sizeof(int32_t))
+        return MOE_ERR_WORKSPACE;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    int32_t* scratch = nullptr;
+    if ((rc = cuda_rc(permute_fixed_scratch(&scratch))) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
+        return rc;
+    rc = cuda_rc(launch_permute(*cfg, topk_ids, offsets, perm_token, dest_row, status, scratch,
+                                st));
+    if (rc != MOE_OK || x_perm == nullptr) return rc;
+    return cuda_rc(launch_gather_rows(*cfg, x, perm_token, offsets, x_perm, st));
+}
+
 MOE_API int moe_grouped_ffn(const moe_cfg* cfg, const uint16_t* x, const uint16_t* x_perm,
                             const int32_t* perm_token, const int32_t* offsets,
                             const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,

@@ -28,6 +28,9 @@ size_t permute_ws_bytes(const moe_cfg& c);
 cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offsets,
                            int32_t* perm_token, int32_t* dest_row, int32_t* status, void* ws,
                            cudaStream_t st);
+// fixed device scratch for moe_permute_noalloc (ints), and its device address
+constexpr int64_t kPermuteFixedScratchInts = 262144;
+cudaError_t permute_fixed_scratch(int32_t** out);
 cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* perm_token,
                                const int32_t* offsets, uint16_t* x_perm, cudaStream_t st);
 

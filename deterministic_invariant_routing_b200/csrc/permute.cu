@@ -10,9 +10,18 @@
 // block's base row per expert) -> placement (per-warp ranks from __match_any_sync in
 // assignment order). All integer, no floating point, no order-dependent atomics (the
 // only atomics are shared-memory histogram increments, whose sum is order-free).
+#include <mutex>
+
 #include "moe_internal.cuh"
 
 namespace moe {
+
+// Fixed scratch of moe_permute_noalloc: the per-block expert histograms live in this
+// file-scope device array instead of a caller workspace. Every GPU that loads the
+// library holds it (1 MiB) until the process exits; all calls share it, and calls that
+// overlap on the GPU race on it.
+static __device__ __align__(256) int32_t g_permute_scratch[kPermuteFixedScratchInts];
+
 namespace {
 
 constexpr int kWarps = 8;                // warps per block
@@ -193,6 +202,27 @@ cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offset
                                                     perm_token);
     }
     return cudaGetLastError();
+}
+
+cudaError_t permute_fixed_scratch(int32_t** out)
+{
+    // In host code g_permute_scratch is only a stand-in symbol, not a device address:
+    // the address is asked of the runtime once per device, with that device current.
+    static std::mutex mu;
+    static int32_t* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_permute_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = addr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* perm_token,

@@ -149,6 +149,28 @@ MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint1
                         void* stream);
 
 /*
+ * moe_permute without a caller workspace. The source pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory at the point where
+ * they dispatch -- for example an engine plug-in that is handed only the tensors of the
+ * current step and must not grow or fragment the engine's memory pool, or plain C code
+ * that has no device allocator of its own. It computes exactly what moe_permute computes
+ * (same arguments minus ws/ws_bytes) and allocates nothing: its per-block histograms live
+ * in one fixed 1 MiB device array inside the library (262144 int32), which every GPU that
+ * loads the library holds until the process exits.
+ *
+ *  Limit: ceil(T*K / 2048) * E <= 262144 (e.g. E = 128 allows T*K <= 4,194,304); larger
+ *         requests return MOE_ERR_WORKSPACE before anything is enqueued.
+ *  The first call on a device looks up the array's device address (once per device, with
+ *  that device current); make that first call before any stream capture.
+ *  All calls share the array and it keeps the last call's contents; nothing in it needs
+ *  to start at zero (every call overwrites what it reads). Calls that overlap on the GPU
+ *  (other streams, other host threads) race on it: serialise them.
+ */
+MOE_API int moe_permute_noalloc(const moe_cfg* cfg, const int32_t* topk_ids, const uint16_t* x,
+                                int32_t* offsets, int32_t* perm_token, int32_t* dest_row,
+                                uint16_t* x_perm, int32_t* status, void* stream);
+
+/*
  * Expert boundary ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 2:
  * gate_and_up -> down; SpecForge PR #1003, experts.py: grouped experts and the
  * always-on shared expert). Grouped SwiGLU GEMMs on the tensor cores:
