@@ -155,3 +155,37 @@ def test_combine_cancellation_order(golden):
     cfg = moe.Config(T=1, H=H, E=8, K=K, I=128)
     out = moe.combine(cfg, y.to(DEV), w.to(DEV), d.to(DEV))
     assert out.float().cpu()[0, 0].item() == c["expect_acc"][0][0]
+
+
+@pytest.mark.parametrize("name,T,n_near", [("tiny", 64, 4), ("dsv_sigmoid", 8192, 410),
+                                           ("qwen3_30b_a3b", 4096, 205)])
+def test_route_injected_near_ties_bit_exact(name, T, n_near):
+    """Tied and 1-ulp-apart choices at the K-th/(K+1)-th boundary (the tiny layer's 4 tied
+    token pairs; 5% of the DeepSeek-style layer's tokens). Experts 2m and 2m+1 share a
+    selection bias, so copying expert a's logit to its partner a^1 ties their choices
+    exactly, and the next float below it puts them within an ulp."""
+    s = synthetic.shape(name, T=T)
+    E, K = s.E, s.K
+    l = synthetic.random_logits(T, E, seed=s.seed + 50, std=2.0).numpy().astype(np.float32)
+    bias = None
+    if s.sel_bias_range is not None:
+        bias = synthetic.uniform_f32(E, s.sel_bias_range, s.seed, "sel_bias").numpy()
+        bias[1::2] = bias[0::2]
+    ids0, _, _ = oracle.route_fp32(l, K, s.score_fn, s.renorm, s.route_scale, sel_bias=bias)
+    rng = np.random.default_rng(s.seed)
+    for i, t in enumerate(rng.choice(T, n_near, replace=False)):
+        a = int(ids0[t, K - 1])
+        b = a ^ 1
+        if b >= E:
+            continue
+        l[t, b] = l[t, a] if i % 2 == 0 else np.nextafter(l[t, a], np.float32(-np.inf))
+    cfg = moe.Config.of(s)
+    _, ids, w = moe.route(cfg, logits=torch.from_numpy(l).to(DEV),
+                          sel_bias=None if bias is None else torch.from_numpy(bias).to(DEV))
+    r_ids, r_w, _ = oracle.route_fp32(l, K, s.score_fn, s.renorm, s.route_scale, sel_bias=bias)
+    assert np.array_equal(ids.cpu().numpy(), r_ids)
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), r_w.view(np.uint32))
+    from helpers import near_tie_count
+    n = near_tie_count(l, s, bias)
+    print(f"\n{name}: {n} of {T} tokens with K-th/(K+1)-th choices within 1 ulp")
+    assert n >= n_near // 2
