@@ -21,10 +21,16 @@ namespace {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// bf16 round-to-nearest-even of two floats packed low/high; a NaN keeps its sign and
+// payload's top bits and is made quiet (the contract's single downcast)
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
-    const __nv_bfloat16 x = __float2bfloat16_rn(a), y = __float2bfloat16_rn(b);
-    return (uint32_t)__bfloat16_as_ushort(x) | ((uint32_t)__bfloat16_as_ushort(y) << 16);
+    auto cvt = [](float f) -> uint32_t {
+        const uint32_t u = __float_as_uint(f);
+        if ((u & 0x7fffffffu) > 0x7f800000u) return (u >> 16) | 0x40u;
+        return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
+    };
+    return cvt(a) | (cvt(b) << 16);
 }
 
 template <int KMAX>

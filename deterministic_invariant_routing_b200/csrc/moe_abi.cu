@@ -140,15 +140,19 @@ cudaError_t router_logits(const moe_cfg& c, const uint16_t* x, const uint16_t* w
     return launch_tc_gemm(p, st);
 }
 
-// gate_up + SwiGLU over grouped rows: h[r] = silu(a_r . W1g^T) * (a_r . W1u^T)
-cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
-                    int rows, const uint16_t* w13, int H, int I, uint16_t* h, int32_t* status,
-                    cudaStream_t st)
+// gate_up + SwiGLU over grouped rows: h[r] = silu(a_r . W1g^T) * (a_r . W1u^T), where
+// a_r is row gather[r] of a when gather is given (the dispatch fused into the GEMM's
+// operand loads) and row r otherwise
+cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, int64_t grouped_rows,
+                    const int32_t* offsets, int groups, int rows, const uint16_t* w13, int H, int I,
+                    uint16_t* h, int32_t* status, cudaStream_t st)
 {
     GemmProblem p{};
     p.epilogue = EPI_SWIGLU;
     p.a = a;
     p.a_rows = a_rows;
+    p.gather_rows = gather;
+    p.a_rows_total = grouped_rows;
     p.b = w13;
     p.b_rows_per_group = 2 * I;
     p.k = H;
@@ -170,6 +174,7 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     p.epilogue = EPI_BF16;
     p.a = h;
     p.a_rows = a_rows;
+    p.a_rows_total = a_rows;
     p.b = w2;
     p.b_rows_per_group = H;
     p.k = I;
@@ -183,7 +188,8 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     return launch_tc_gemm(p, st);
 }
 
-int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm, const int32_t* offsets,
+int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm,
+             const int32_t* perm_token, const int32_t* offsets,
              const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s, const uint16_t* w2_s,
              uint16_t* y, uint16_t* y_shared, int32_t* status, void* ws, void* const* ev,
              cudaStream_t st)
@@ -191,7 +197,11 @@ int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm, const 
     const FfnLayout L = ffn_layout(c);
     const int64_t A = (int64_t)c.T * c.K;
     uint16_t* h = at<uint16_t>(ws, L.h);
-    int rc = cuda_rc(gate_up(x_perm, A, offsets, c.E, 0, w13, c.H, c.I, h, status, st));
+    int rc = x_perm != nullptr
+                 ? cuda_rc(gate_up(x_perm, A, nullptr, A, offsets, c.E, 0, w13, c.H, c.I, h, status,
+                                   st))
+                 : cuda_rc(gate_up(x, c.T, perm_token, A, offsets, c.E, 0, w13, c.H, c.I, h, status,
+                                   st));
     if (rc != MOE_OK) return rc;
     if ((rc = rec(ev, 4, st)) != MOE_OK) return rc;
     rc = cuda_rc(down(h, A, offsets, c.E, 0, w2, c.H, c.I, y, status, st));
@@ -199,7 +209,8 @@ int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm, const 
     if ((rc = rec(ev, 5, st)) != MOE_OK) return rc;
     if (c.I_shared > 0 && w13_s != nullptr) {
         uint16_t* h_s = at<uint16_t>(ws, L.h_s);
-        rc = cuda_rc(gate_up(x, c.T, nullptr, 1, c.T, w13_s, c.H, c.I_shared, h_s, status, st));
+        rc = cuda_rc(gate_up(x, c.T, nullptr, c.T, nullptr, 1, c.T, w13_s, c.H, c.I_shared, h_s,
+                             status, st));
         if (rc != MOE_OK) return rc;
         rc = cuda_rc(down(h_s, c.T, nullptr, 1, c.T, w2_s, c.H, c.I_shared, y_shared, status, st));
         if (rc != MOE_OK) return rc;
@@ -324,18 +335,16 @@ MOE_API int moe_grouped_ffn(const moe_cfg* cfg, const uint16_t* x, const uint16_
     if (shared && (x == nullptr || w13_s == nullptr || w2_s == nullptr || y_shared == nullptr ||
                    !aligned16(x) || !aligned16(w13_s) || !aligned16(w2_s) || !aligned16(y_shared)))
         return MOE_ERR_ARG;
-    if (x_perm == nullptr) {
-        if (perm_token == nullptr || x == nullptr) return MOE_ERR_ARG;
-        return MOE_ERR_UNIMPLEMENTED;
-    }
-    if (!aligned16(x_perm)) return MOE_ERR_ARG;
+    if (x_perm == nullptr && (perm_token == nullptr || x == nullptr || !aligned16(x)))
+        return MOE_ERR_ARG;
+    if (x_perm != nullptr && !aligned16(x_perm)) return MOE_ERR_ARG;
     if (ws == nullptr || ws_bytes < ffn_layout(*cfg).total) return MOE_ERR_WORKSPACE;
     if (cfg->T == 0) return MOE_OK;
     if ((rc = check_device()) != MOE_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
         return rc;
-    return ffn_impl(*cfg, x, x_perm, offsets, w13, w2, shared ? w13_s : nullptr,
+    return ffn_impl(*cfg, x, x_perm, perm_token, offsets, w13, w2, shared ? w13_s : nullptr,
                     shared ? w2_s : nullptr, y, y_shared, status, ws, nullptr, st);
 }
 
@@ -402,9 +411,10 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
     rc = cuda_rc(launch_permute(c, ids, offs, perm_token, dest_row, status,
                                 at<void>(ws, L.perm_ws), st));
     if (rc != MOE_OK) return rc;
+    // materialised dispatch: the gather fused into the GEMM's operand loads is slower here
     if ((rc = cuda_rc(launch_gather_rows(c, x, perm_token, offs, x_perm, st))) != MOE_OK) return rc;
     if ((rc = rec(ev, 3, st)) != MOE_OK) return rc;
-    rc = ffn_impl(c, x, x_perm, offs, w13, w2, shared ? w13_s : nullptr, shared ? w2_s : nullptr,
+    rc = ffn_impl(c, x, x_perm, perm_token, offs, w13, w2, shared ? w13_s : nullptr, shared ? w2_s : nullptr,
                   y, y_s, status, at<void>(ws, L.ffn), ev, st);
     if (rc != MOE_OK) return rc;
     rc = cuda_rc(launch_combine(c, y, w, dest_row, y_s, token_mask, out, st));

@@ -46,6 +46,8 @@ struct GemmProblem {
     int epilogue;            // GemmEpilogue
     const uint16_t* a;       // A [a_rows, k] bf16 (row-major, K-major)
     int64_t a_rows;          // rows of the A buffer (TMA bound)
+    const int32_t* gather_rows;  // grouped row r reads A row gather_rows[r] (NULL: row r)
+    int64_t a_rows_total;    // grouped rows (bound of offsets[groups])
     const uint16_t* b;       // B [groups * b_rows_per_group, k] bf16
     int b_rows_per_group;    // SWIGLU: 2*I (gate rows then up rows); else N
     int k;                   // reduction length (multiple of 64)
@@ -60,6 +62,7 @@ struct GemmProblem {
 };
 
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st);
+cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st);
 
 // device facts
 int num_sms();

@@ -150,7 +150,8 @@ __global__ void __launch_bounds__(kWarps * 32) place_kernel(const int32_t* __res
     }
 }
 
-// x_perm[r, :] = x[perm_token[r], :] for r < offsets[E]; one warp per row, 16 B per lane
+// x_perm[r, :] = x[perm_token[r], :] for r < offsets[E]; one warp per row, 16 B per lane,
+// up to 8 loads per lane in flight before the stores
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
                                                      const int32_t* __restrict__ perm_token,
                                                      const int32_t* __restrict__ offsets, int E,
@@ -165,7 +166,15 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
         const int64_t t = perm_token[r];
         const uint4* src = x + t * vec_per_row;
         uint4* dst = x_perm + r * vec_per_row;
-        for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < vec_per_row) buf[u] = src[v0 + 32 * u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < vec_per_row) dst[v0 + 32 * u] = buf[u];
+        }
     }
 }
 

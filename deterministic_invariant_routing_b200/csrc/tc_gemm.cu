@@ -27,181 +27,14 @@
 // returns.
 #include <cuda_bf16.h>
 
-#include "moe_internal.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int BM = 128;                   // rows per tile = UMMA M = TMEM lanes
-constexpr int BK = 64;                    // k-block: one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;
 constexpr uint32_t kABytes = BM * BK * 2;  // 16 KiB per stage
-constexpr long long kTimeoutCycles = 2000000000LL;  // about a second at B200 clocks
-constexpr int kSmemBudget = 196608;        // bytes for the operand ring
-
-// ------------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Wait for the phase of parity `parity` of `bar` to complete. Gives up (returns false)
-// after about a second, or as soon as another role raised the abort flag.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status, bool honour_abort = true)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0u) {
-            if (honour_abort && *abort_flag) return false;
-            if (clock64() - t0 > kTimeoutCycles) {
-                if (!*abort_flag) {
-                    *abort_flag = 1;
-                    status_add(status, MOE_ST_PIPE_TIMEOUT, 1);
-                }
-                return false;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before()
-{
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after()
-{
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     dst_smem),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
-                 "r"(ncols)
-                 : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate, M=128, N=BN, K=16
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// arrive on `bar` once every tcgen05 op issued so far by this thread has completed
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane, waited for in the same asm so
-// no use of the registers can be scheduled before the data lands
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
-        "[%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with 128-byte
-// swizzling: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), the
-// leading byte offset unused for this layout (1), descriptor version 1, swizzle mode 2.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
-{
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3fffu);
-    d |= (uint64_t)1u << 16;
-    d |= (uint64_t)(1024u >> 4) << 32;
-    d |= (uint64_t)1u << 46;
-    d |= (uint64_t)2u << 61;
-    return d;
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t make_idesc(int m, int n)
-{
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-           ((uint32_t)(m >> 4) << 24);
-}
-
-// bf16 round-to-nearest-even of two floats packed low/high (NaN stays NaN, quieted)
-__device__ __forceinline__ uint32_t bf16x2_rne(float lo, float hi)
-{
-    auto cvt = [](float f) -> uint32_t {
-        uint32_t u = __float_as_uint(f);
-        if ((u & 0x7fffffffu) > 0x7f800000u) return (u >> 16) | 0x40u;
-        return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
-    };
-    return cvt(lo) | (cvt(hi) << 16);
-}
 
 struct TcArgs {
     int k_blocks;
@@ -453,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int h2 = 0; h2 < 2; ++h2) {
                             const float gv = __uint_as_float(g[2 * j + h2]);
                             const float uv = __uint_as_float(u[2 * j + h2]);
-                            hv[h2] = gv / (1.0f + expf(-gv)) * uv;
+                            hv[h2] = swiglu(gv, uv);
                         }
                         pk[j] = bf16x2_rne(hv[0], hv[1]);
                     }
@@ -520,41 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 2-D bf16 tensor [rows, cols] (cols contiguous), box = 64 columns x box_rows rows,
-// 128-byte swizzle, zero fill outside the tensor
-bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int EPI, int BN>
 cudaError_t launch_variant(const GemmProblem& p, cudaStream_t st)
 {
@@ -589,7 +387,7 @@ cudaError_t launch_variant(const GemmProblem& p, cudaStream_t st)
     a.n_valid = p.n;
     a.bias = p.bias;
     a.status = p.status;
-    const int64_t rows_total = p.offsets ? p.a_rows : p.rows;
+    const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
     const int64_t max_tiles = ((rows_total + BM - 1) / BM + groups) * a.n_tiles;
     int grid = num_sms();
     if (max_tiles < grid) grid = (int)max_tiles;
@@ -603,15 +401,8 @@ cudaError_t launch_variant(const GemmProblem& p, cudaStream_t st)
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st)
 {
     if (p.k % BK != 0) return cudaErrorInvalidValue;
-    if (p.epilogue == EPI_SWIGLU) {
-        if (p.n % 128 != 0) return cudaErrorInvalidValue;
-        return launch_variant<EPI_SWIGLU, 256>(p, st);
-    }
-    if (p.epilogue == EPI_BF16) {
-        if (p.n % 256 == 0) return launch_variant<EPI_BF16, 256>(p, st);
-        if (p.n % 128 == 0) return launch_variant<EPI_BF16, 128>(p, st);
-        return cudaErrorInvalidValue;
-    }
+    // the expert products run on CTA pairs (tc_gemm2.cu)
+    if (p.epilogue == EPI_SWIGLU || p.epilogue == EPI_BF16) return launch_tc_gemm_pair(p, st);
     // fp32 epilogue (router logits): N = next power of two >= E, at least 32, at most 256
     if (p.n <= 32) return launch_variant<EPI_F32, 32>(p, st);
     if (p.n <= 64) return launch_variant<EPI_F32, 64>(p, st);

@@ -1,0 +1,509 @@
+// Grouped GEMM on CTA pairs: tcgen05.mma.cta_group::2 (M = 256 rows per tile split over
+// the two CTAs of a cluster), TMA operand loads, TMEM accumulators. Used for the expert
+// products -- gate_up with the SwiGLU epilogue and down -- of "DSV4 Flash MoE
+// Train-Inference Consistency Roadmap", Problem 2 (gate_and_up -> down) and SpecForge
+// PR #1003 (grouped experts, the always-on shared expert as one more group).
+//
+// Why a pair: one UMMA of M=128, N=256, K=16 reads 12 KiB of operands from shared memory
+// per 128 tensor cycles, and the TMA ring writes as much again -- more than one SM's
+// shared-memory bandwidth. With cta_group::2 each SM holds its own 128 rows of A and only
+// half of B's columns, so each SM moves 8 KiB per 128 cycles each way.
+//
+//   leader (even CTA)  A rows [r0, r0+128)       B columns [0, N/2)    TMEM rows r0..
+//   peer   (odd CTA)   A rows [r0+128, r0+256)   B columns [N/2, N)    TMEM rows r0+128..
+//
+// For the SwiGLU product the pair's N = 256 is 128 gate columns (the leader's B half)
+// followed by the 128 matching up columns (the peer's B half), so every CTA's accumulator
+// row holds gate and up of the same 128 intermediate columns.
+//
+// Batch invariance: the tile shape (256 x N), the instruction shape and the K order
+// (k-blocks of 64 in increasing k, four K=16 steps each) depend only on the GEMM's (N, K);
+// rows past the group's end are computed and never stored; no split-K, no atomics.
+//
+// Protocol (per k-block stage s): both CTAs wait on their own empty[s], load their A and
+// B halves with .cta_group::2 TMA whose completion is counted on the LEADER's full[s]
+// (the leader posts the byte count of both CTAs); the leader's single MMA thread waits on
+// full[s], issues the pair MMAs and commits to empty[s] of both CTAs (multicast commit).
+// Accumulators: the commit of the last k-block arrives on tfull[a] of both CTAs; each
+// CTA's epilogue drains its own TMEM rows and arrives on the leader's tempty[a] (256
+// arrivals). Every wait is bounded and a give-up is recorded in MOE_ST_PIPE_TIMEOUT.
+#include <cuda_bf16.h>
+
+#include "tc_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int PM = 256;                     // rows per pair tile
+constexpr int HM = 128;                     // rows per CTA = TMEM lanes
+constexpr int kThreads2 = 192;
+constexpr uint32_t kA2Bytes = HM * BK * 2;  // 16 KiB per stage
+constexpr uint16_t kPairMask = 0x3;
+
+struct PairArgs {
+    int k_blocks;
+    int n_tiles;
+    int groups;
+    const int32_t* offsets;
+    int rows;
+    int b_rows_per_group;
+    int half_rows;  // SWIGLU: rows between a gate row and its up row in B
+    const int32_t* gather_rows;  // A row r is row gather_rows[r] of the A tensor, or NULL
+    const uint16_t* a;           // the A tensor (read directly by a gather)
+    int k;                       // its row length
+    void* out;
+    int64_t ldo;
+    int32_t* status;
+};
+
+template <int EPI, int NP>
+struct Cfg2 {
+    static_assert(NP == 128 || NP == 256, "pair N");
+    static constexpr uint32_t kBBytes = (uint32_t)(NP / 2) * BK * 2;  // this CTA's half of B
+    static constexpr uint32_t kStageBytes = kA2Bytes + kBBytes;
+    static constexpr int kStages0 = kSmemBudget / (int)kStageBytes;
+    static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+    static constexpr uint32_t kTmemCols = 2 * NP;
+    static constexpr int kBars = 2 * kStages + 5;
+    static size_t smem_bytes(int groups)
+    {
+        return 1024 + (size_t)kStages * kStageBytes + kBars * 8 + 16 +
+               (size_t)2 * (groups + 1) * sizeof(int32_t) + HM * sizeof(int32_t);
+    }
+};
+
+struct PairTile {
+    int g, n;
+    int64_t row0, row_end;  // row0: the pair tile's first row
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(int t, int n_tiles, int groups,
+                                                     const int32_t* prefix, const int32_t* offs)
+{
+    PairTile ti;
+    const int mt = t / n_tiles;
+    ti.n = t - mt * n_tiles;
+    int lo = 0, hi = groups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= mt) lo = mid;
+        else hi = mid - 1;
+    }
+    ti.g = lo;
+    ti.row0 = (int64_t)offs[lo] + (int64_t)(mt - prefix[lo]) * PM;
+    ti.row_end = offs[lo + 1];
+    return ti;
+}
+
+template <int EPI, int NP, bool GATHER>
+__global__ void __launch_bounds__(kThreads2, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, PairArgs args)
+{
+    using C = Cfg2<EPI, NP>;
+    constexpr int S = C::kStages;
+    constexpr uint32_t kIdesc = make_idesc(PM, NP);
+    constexpr int kBRows = NP / 2;  // B rows per CTA per stage
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    uint8_t* base = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sA0 = smem_u32(base);
+    const uint32_t sB0 = sA0 + S * kA2Bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * C::kStageBytes);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(S + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (uint32_t)(2 * S + 4);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(bars + C::kBars);  // [0] tmem, [1] abort
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    int32_t* prefix = reinterpret_cast<int32_t*>(misc + 4);
+    int32_t* offs = prefix + (args.groups + 1);
+    int32_t* gather_tok = offs + (args.groups + 1);  // [HM] source rows of the current tile
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = args.groups;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), GATHER ? 3 : 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 2 * 4 * 32);
+        }
+        mbar_init(drain_bar, 1);
+        misc[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
+    if (warp == 2) {
+        auto row_off = [&](int g) -> int {
+            return args.offsets ? args.offsets[g] : (g == 0 ? 0 : args.rows);
+        };
+        const int per = (G + 31) / 32;
+        const int beg = lane * per < G ? lane * per : G;
+        const int end = beg + per < G ? beg + per : G;
+        int sum = 0;
+        for (int g = beg; g < end; ++g) {
+            const int r0 = row_off(g);
+            offs[g] = r0;
+            sum += (row_off(g + 1) - r0 + PM - 1) / PM;
+        }
+        if (lane == 0) offs[G] = row_off(G);
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        int run = incl - sum;
+        for (int g = beg; g < end; ++g) {
+            prefix[g] = run;
+            run += (row_off(g + 1) - row_off(g) + PM - 1) / PM;
+        }
+        if (lane == 31) prefix[G] = incl;
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers and TMEM of both CTAs ready before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = misc[0];
+    const int total = prefix[G] * args.n_tiles;
+
+    if (warp == 0 && !GATHER) {
+        // -------------------------------------------------------------- TMA producer
+        // one thread: A and B tiles by TMA, bytes counted on the leader's full[s]
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_phase = 0;
+            for (int t = cluster; t < total && !*abort_flag; t += nclusters) {
+                const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+                const int arow = (int)ti.row0 + (int)rank * HM;
+                const int brow = (EPI == EPI_SWIGLU)
+                                     ? ti.g * args.b_rows_per_group +
+                                           (leader ? 0 : args.half_rows) + ti.n * kBRows
+                                     : ti.g * args.b_rows_per_group + ti.n * NP +
+                                           (int)rank * kBRows;
+                bool ok = true;
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = mapa_shared(full_bar(stage), 0);
+                    if (leader) mbar_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+                    tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, kb * BK, arow, fb);
+                    tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kb * BK, brow, fb);
+                    armed |= 1u << stage;
+                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+            if (*abort_flag && leader) {
+                for (int s = 0; s < S; ++s)
+                    if (armed & (1u << s))
+                        wait_bounded(full_bar(s), (armed_phase >> s) & 1u, abort_flag,
+                                     args.status, false);
+            }
+        }
+    } else if (warp == 0) {
+        // -------------------------------------------------------------- gathering producer
+        // B (and A without a gather): TMA issued by lane 0, bytes counted on the leader's
+        // full[s]. With a gather, A row r of this CTA's 128 is token row gather_rows[r] of
+        // the A tensor: each lane copies 4 rows with 16-byte cp.async, writing the 128-byte
+        // swizzle itself; kLag stages later it waits for those copies, fences them into
+        // the async proxy, and lane 0 arrives once for the CTA on the leader's full[s].
+        // Loop decisions are lane 0's, broadcast, so the warp stays converged.
+        constexpr int kLag = S - 2;
+        int stage = 0, sig_stage = 0, pending = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_phase = 0;
+        const uint32_t fb0 = mapa_shared(full_bar(0), 0);
+        auto signal_oldest = [&](int keep) {
+            // all but `keep` of this lane's newest copy groups have landed
+            if (keep >= kLag) cp_async_wait_group<kLag>();
+            else cp_async_wait_all();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(fb0 + 8u * (uint32_t)sig_stage);
+            if (++sig_stage == S) sig_stage = 0;
+            --pending;
+        };
+        for (int t = cluster; t < total; t += nclusters) {
+            if (!__shfl_sync(0xffffffffu, lane == 0 ? !*abort_flag : 0, 0)) break;
+            const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+            const int arow = (int)ti.row0 + (int)rank * HM;
+            const int brow = (EPI == EPI_SWIGLU)
+                                 ? ti.g * args.b_rows_per_group + (leader ? 0 : args.half_rows) +
+                                       ti.n * kBRows
+                                 : ti.g * args.b_rows_per_group + ti.n * NP + (int)rank * kBRows;
+            if (GATHER) {
+                // source token of each of this CTA's 128 rows; rows past the group's end
+                // repeat its last row (computed, never stored)
+                const int64_t last = ti.row_end - 1;
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t r = (int64_t)arow + 32 * i + lane;
+                    gather_tok[32 * i + lane] = args.gather_rows[r < ti.row_end ? r : last];
+                }
+                __syncwarp();
+            }
+            int ok = 1;
+            for (int kb = 0; kb < args.k_blocks; ++kb) {
+                if (lane == 0)
+                    ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const uint32_t fb = fb0 + 8u * (uint32_t)stage;
+                const uint32_t sa = sA0 + (uint32_t)stage * kA2Bytes;
+                if (lane == 0) {
+                    if (leader)
+                        mbar_expect_tx(full_bar(stage),
+                                       GATHER ? 2 * C::kBBytes : 2 * C::kStageBytes);
+                    if (!GATHER) tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
+                    tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kb * BK, brow, fb);
+                    armed |= 1u << stage;
+                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                }
+                if (GATHER) {
+                    // each instruction copies 4 whole 128-byte rows: 8 lanes per row, one
+                    // 16-byte chunk each, stored at its swizzled place
+                    const int c = lane & 7;
+#pragma unroll 8
+                    for (int i = 0; i < HM / 4; ++i) {
+                        const int r = 4 * i + (lane >> 3);  // row within this CTA's 128
+                        const uint16_t* g =
+                            args.a + (int64_t)gather_tok[r] * args.k + kb * BK + c * 8;
+                        cp_async_16(sa + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)), g);
+                    }
+                    cp_async_commit();
+                    if (++pending > kLag) signal_oldest(kLag);
+                }
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+        if (GATHER)
+            while (pending > 0) signal_oldest(0);
+        if (lane == 0 && *abort_flag && leader) {
+            for (int s = 0; s < S; ++s)
+                if (armed & (1u << s))
+                    wait_bounded(full_bar(s), (armed_phase >> s) & 1u, abort_flag, args.status,
+                                 false);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------------------------------------------------- MMA issuer
+            int stage = 0;
+            uint32_t phase = 0;
+            int i = 0;
+            for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
+                const int acc = i & 1;
+                if (!wait_bounded(tempty_bar(acc), (((uint32_t)i >> 1) & 1u) ^ 1u, abort_flag,
+                                  args.status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NP);
+                bool ok = true;
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!wait_bounded(full_bar(stage), phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(sA0 + (uint32_t)stage * kA2Bytes);
+                    const uint64_t bd = sw128_desc(sB0 + (uint32_t)stage * C::kBBytes);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
+                                      kIdesc, (kb | k) != 0 ? 1u : 0u);
+                    mma_commit_pair_mc(empty_bar(stage), kPairMask);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair_mc(tfull_bar(acc), kPairMask);
+            }
+            mma_commit_pair(drain_bar);
+            wait_bounded(drain_bar, 0u, abort_flag, args.status, false);
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+        const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
+        int i = 0;
+        for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
+            const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+            const int acc = i & 1;
+            int ok = 1;
+            if (lane == 0)
+                ok = wait_bounded(tfull_bar(acc), ((uint32_t)i >> 1) & 1u, abort_flag, args.status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * NP);
+            const int64_t grow = ti.row0 + (int64_t)rank * HM + row;
+            const bool valid = grow < ti.row_end;
+            uint16_t* out = static_cast<uint16_t*>(args.out);
+            if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < NP / 2; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(tbase + (uint32_t)c, g);
+                    tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float hv[2];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const float gv = __uint_as_float(g[2 * j + h2]);
+                            const float uv = __uint_as_float(u[2 * j + h2]);
+                            hv[h2] = swiglu(gv, uv);
+                        }
+                        pk[j] = bf16x2_rne(hv[0], hv[1]);
+                    }
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            out + grow * args.ldo + (int64_t)ti.n * (NP / 2) + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                                pk[4 * v + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < NP; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + (uint32_t)c, r);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pk[j] = bf16x2_rne(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo +
+                                                              (int64_t)ti.n * NP + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                                pk[4 * v + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // the peer's last remote arrivals and the leader's MMAs are done
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    }
+}
+
+template <int EPI, int NP, bool GATHER>
+cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
+{
+    using C = Cfg2<EPI, NP>;
+    auto kernel = tc_gemm_pair_kernel<EPI, NP, GATHER>;
+    const int groups = p.offsets ? p.groups : 1;
+    const size_t smem = C::smem_bytes(groups);
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    static bool attr_set[64] = {};
+    static int max_clusters[64] = {};
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads2, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+        if (err != cudaSuccess) return err;
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.dynamicSmemBytes = C::smem_bytes(1025);
+        int n = 0;
+        err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+        if (err != cudaSuccess) return err;
+        max_clusters[dev] = n > 0 ? n : 1;
+        cfg.dynamicSmemBytes = smem;
+        attr_set[dev] = true;
+    }
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, p.b, (int64_t)groups * p.b_rows_per_group, p.k, NP / 2))
+        return cudaErrorInvalidValue;
+    PairArgs a;
+    a.k_blocks = p.k / BK;
+    a.n_tiles = (EPI == EPI_SWIGLU) ? p.n / (NP / 2) : p.n / NP;
+    a.groups = groups;
+    a.offsets = p.offsets;
+    a.rows = p.rows;
+    a.b_rows_per_group = p.b_rows_per_group;
+    a.half_rows = (EPI == EPI_SWIGLU) ? p.n : 0;
+    a.gather_rows = p.gather_rows;
+    a.a = p.a;
+    a.k = p.k;
+    a.out = p.out;
+    a.ldo = p.ldo;
+    a.status = p.status;
+    const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
+    const int64_t max_tiles = ((rows_total + PM - 1) / PM + groups) * a.n_tiles;
+    int64_t clusters = max_clusters[dev];
+    if (max_tiles < clusters) clusters = max_tiles;
+    if (clusters < 1) clusters = 1;
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, a);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st)
+{
+    if (p.k % BK != 0) return cudaErrorInvalidValue;
+    if (p.epilogue == EPI_SWIGLU) {
+        if (p.n % 128 != 0) return cudaErrorInvalidValue;
+        if (p.gather_rows) return launch_pair_variant<EPI_SWIGLU, 256, true>(p, st);
+        return launch_pair_variant<EPI_SWIGLU, 256, false>(p, st);
+    }
+    if (p.gather_rows) return cudaErrorInvalidValue;
+    if (p.epilogue == EPI_BF16) {
+        if (p.n % 256 == 0) return launch_pair_variant<EPI_BF16, 256, false>(p, st);
+        if (p.n % 128 == 0) return launch_pair_variant<EPI_BF16, 128, false>(p, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

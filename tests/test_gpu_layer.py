@@ -101,6 +101,11 @@ def check_layer(name, T, n_sample=16, keep=None, report=None):
     if mask_np is not None:
         assert np.all(bits(r["out"])[mask_np == 0] == 0)
 
+    # the gather fused into the GEMM's operand loads gives the same expert outputs
+    y_g, ys_g = moe.grouped_ffn(cfg, d["x"], None, r["perm_token"], r["offsets"], d["w13"],
+                                d["w2"], d["w13_s"], d["w2_s"])
+    assert np.array_equal(bits(y_g[:n_rows]), bits(r["y"][:n_rows]))
+
     # the one-call forward is the same computation
     out1, b = moe.forward(cfg, d["x"], d["w_router"], d["w13"], d["w2"],
                           logit_bias=d["logit_bias"], sel_bias=d["sel_bias"], token_mask=mask,
