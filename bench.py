@@ -57,19 +57,24 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha(rel):
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(rels):
+    """Hash of the kernel's source files (a list of repo-relative paths)."""
+    h = hashlib.sha256()
+    for rel in rels:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel_key):
-    """DRAM bytes per launch of a kernel from a committed ncu summary, or None when the
-    kernel's source changed since the counters were taken."""
+    """DRAM bytes per launch of a kernel from a committed ncu summary
+    (profiles/ncu_traffic.json), or None when the kernel's sources changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
-        if rec["source_sha"] != source_sha(rec["source"]):
+        if rec["source_sha"] != source_sha(rec["sources"]):
             return None
         return rec["bytes_per_launch"]
     except Exception:

@@ -294,7 +294,7 @@ MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint1
         return rc;
     rc = cuda_rc(launch_permute(*cfg, topk_ids, offsets, perm_token, dest_row, status, ws, st));
     if (rc != MOE_OK || x_perm == nullptr) return rc;
-    return cuda_rc(launch_gather_rows(*cfg, x, perm_token, offsets, x_perm, st));
+    return cuda_rc(launch_gather_rows(*cfg, x, dest_row, x_perm, st));
 }
 
 MOE_API int moe_permute_noalloc(const moe_cfg* cfg, const int32_t* topk_ids, const uint16_t* x,
@@ -318,7 +318,7 @@ MOE_API int moe_permute_noalloc(const moe_cfg* cfg, const int32_t* topk_ids, con
     rc = cuda_rc(launch_permute(*cfg, topk_ids, offsets, perm_token, dest_row, status, scratch,
                                 st));
     if (rc != MOE_OK || x_perm == nullptr) return rc;
-    return cuda_rc(launch_gather_rows(*cfg, x, perm_token, offsets, x_perm, st));
+    return cuda_rc(launch_gather_rows(*cfg, x, dest_row, x_perm, st));
 }
 
 MOE_API int moe_grouped_ffn(const moe_cfg* cfg, const uint16_t* x, const uint16_t* x_perm,
@@ -412,7 +412,7 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
                                 at<void>(ws, L.perm_ws), st));
     if (rc != MOE_OK) return rc;
     // materialised dispatch: the gather fused into the GEMM's operand loads is slower here
-    if ((rc = cuda_rc(launch_gather_rows(c, x, perm_token, offs, x_perm, st))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(launch_gather_rows(c, x, dest_row, x_perm, st))) != MOE_OK) return rc;
     if ((rc = rec(ev, 3, st)) != MOE_OK) return rc;
     rc = ffn_impl(c, x, x_perm, perm_token, offs, w13, w2, shared ? w13_s : nullptr, shared ? w2_s : nullptr,
                   y, y_s, status, at<void>(ws, L.ffn), ev, st);

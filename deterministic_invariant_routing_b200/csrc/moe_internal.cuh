@@ -31,8 +31,9 @@ cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offset
 // fixed device scratch for moe_permute_noalloc (ints), and its device address
 constexpr int64_t kPermuteFixedScratchInts = 262144;
 cudaError_t permute_fixed_scratch(int32_t** out);
-cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* perm_token,
-                               const int32_t* offsets, uint16_t* x_perm, cudaStream_t st);
+// x_perm[dest_row[t, j]] = x[t] for every routed assignment (token-major)
+cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* dest_row,
+                               uint16_t* x_perm, cudaStream_t st);
 
 // combine
 cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,

@@ -150,30 +150,33 @@ __global__ void __launch_bounds__(kWarps * 32) place_kernel(const int32_t* __res
     }
 }
 
-// x_perm[r, :] = x[perm_token[r], :] for r < offsets[E]; one warp per row, 16 B per lane,
-// up to 8 loads per lane in flight before the stores
+// x_perm[dest_row[t, j], :] = x[t, :] for every routed (t, j): one warp per token, which
+// reads the token's row once (8 vectors of 16 B per lane in flight) and writes its K
+// copies -- token-major, so each row of x leaves DRAM once.
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
-                                                     const int32_t* __restrict__ perm_token,
-                                                     const int32_t* __restrict__ offsets, int E,
-                                                     int64_t max_rows, int vec_per_row,
+                                                     const int32_t* __restrict__ dest_row, int T,
+                                                     int K, int vec_per_row,
                                                      uint4* __restrict__ x_perm)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t rows = offsets[E];
     const int64_t wpb = blockDim.x >> 5;
-    for (int64_t r = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); r < rows && r < max_rows;
-         r += (int64_t)gridDim.x * wpb) {
-        const int64_t t = perm_token[r];
+    for (int64_t t = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); t < T;
+         t += (int64_t)gridDim.x * wpb) {
+        const int32_t my_dest = lane < K ? dest_row[t * K + lane] : -1;
         const uint4* src = x + t * vec_per_row;
-        uint4* dst = x_perm + r * vec_per_row;
         for (int v0 = lane; v0 < vec_per_row; v0 += 32 * 8) {
             uint4 buf[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 if (v0 + 32 * u < vec_per_row) buf[u] = src[v0 + 32 * u];
+            for (int j = 0; j < K; ++j) {
+                const int32_t d = __shfl_sync(0xffffffffu, my_dest, j);
+                if (d < 0) continue;
+                uint4* dst = x_perm + (int64_t)d * vec_per_row;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (v0 + 32 * u < vec_per_row) dst[v0 + 32 * u] = buf[u];
+                for (int u = 0; u < 8; ++u)
+                    if (v0 + 32 * u < vec_per_row) dst[v0 + 32 * u] = buf[u];
+            }
         }
     }
 }
@@ -234,17 +237,16 @@ cudaError_t permute_fixed_scratch(int32_t** out)
     return cudaSuccess;
 }
 
-cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* perm_token,
-                               const int32_t* offsets, uint16_t* x_perm, cudaStream_t st)
+cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* dest_row,
+                               uint16_t* x_perm, cudaStream_t st)
 {
-    const int64_t A = (int64_t)c.T * c.K;
-    if (A == 0) return cudaSuccess;
+    if (c.T == 0) return cudaSuccess;
     const int vec = c.H / 8;
-    int64_t blocks = (A + 7) / 8;
+    int64_t blocks = ((int64_t)c.T + 7) / 8;
     const int64_t cap = (int64_t)num_sms() * 16;
     if (blocks > cap) blocks = cap;
-    gather_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(x),
-                                                    perm_token, offsets, c.E, A, vec,
+    gather_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), dest_row,
+                                                    c.T, c.K, vec,
                                                     reinterpret_cast<uint4*>(x_perm));
     return cudaGetLastError();
 }
