@@ -132,6 +132,36 @@ class ClockSampler:
                 "sm_max_mhz": mx or None, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def dist_env():
+    """(rank, world size, local rank) from the torchrun environment (1 process if unset)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(v, dev, world):
+    """The max of a per-rank number over all ranks (the slowest rank's time)."""
+    if world == 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_inputs(s, rank, device):
+    """Each rank is a replica: the same weights everywhere, its own tokens."""
+    from deterministic_invariant_routing_b200 import synthetic
+    weights = synthetic.make_weights(s, device=device)
+    x = synthetic.make_tokens(s, s.T, seed=s.seed + 1000 * rank, device=device)
+    return weights, x
+
+
+def job_tokens_per_s(T_per_rank, world, ms_max):
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return T_per_rank * world / (ms_max * 1e-3)
+
+
 def layer_work(s, n_touched):
     """Algorithmic FLOPs and bytes of one layer forward (intermediates excluded)."""
     T, H, E, K, I, Is = s.T, s.H, s.E, s.K, s.I, s.I_shared
@@ -175,7 +205,7 @@ def run_reference(a):
     """The correctness reference (the CPU oracle, as it stands) on the host cores; each
     step is a bounded token sample, the whole run about 90 s."""
     from deterministic_invariant_routing_b200 import synthetic
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = dist_env()
     if rank != 0:
         return
     s, d = synthetic.make_layer(a.workload, T=a.T, device="cpu")
@@ -219,9 +249,7 @@ def main():
 
     from deterministic_invariant_routing_b200 import moe, synthetic
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -230,8 +258,7 @@ def main():
                                 device_id=dev)
 
     s = synthetic.shape(a.workload, T=a.T)
-    weights = synthetic.make_weights(s, device=dev)
-    x = synthetic.make_tokens(s, s.T, seed=s.seed + 1000 * rank, device=dev)
+    weights, x = replica_inputs(s, rank, dev)
     cfg = moe.Config.of(s)
     layer = moe.MoELayer(cfg, weights)
 
@@ -248,11 +275,7 @@ def main():
         torch.cuda.synchronize()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev, world)
 
     K = a.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
@@ -306,7 +329,7 @@ def main():
     clocks = clk.summary()
     line = {
         "metric": "MoE-layer tokens/s (bf16, batch-invariant)",
-        "value": s.T * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "value": job_tokens_per_s(s.T, world, ms), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(s, world),
@@ -320,7 +343,7 @@ def main():
                            "peaks": f"{pk_src}: {peak} TFLOP/s bf16 sustained, "
                                     f"{pk['hbm_gbs']} GB/s"},
         "stage_ms": stages,
-        "e2e": {"value": s.T * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(s.T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},
         "gpu_launches": K * (9 + (2 if s.I_shared else 0)),
         "clocks": clocks,
