@@ -59,6 +59,8 @@ SIGNATURES = {
     "moe_combine": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          _SZ, _P, _P]),
+    "moe_forward_host_workspace_bytes": (_SZ, [_CFG, _I]),
+    "moe_forward_host": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_abi_version": (_I, []),
 }

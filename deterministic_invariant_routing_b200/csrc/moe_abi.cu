@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -218,6 +220,119 @@ int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm,
     return rec(ev, 6, st);
 }
 
+int check_forward_args(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                       const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
+                       const uint16_t* w2_s, const uint16_t* out, const int32_t* status)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (x == nullptr || w_router == nullptr || w13 == nullptr || w2 == nullptr || out == nullptr ||
+        status == nullptr)
+        return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) ||
+        !aligned16(out))
+        return MOE_ERR_ARG;
+    if (cfg->I_shared > 0 &&
+        (w13_s == nullptr || w2_s == nullptr || !aligned16(w13_s) || !aligned16(w2_s)))
+        return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+// the layer on device tensors; status is not cleared (callers clear it once)
+int forward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* w_router,
+                 const float* logit_bias, const float* sel_bias, const uint8_t* token_mask,
+                 const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
+                 const uint16_t* w2_s, uint16_t* out, float* logits, int32_t* topk_ids,
+                 float* topk_w, int32_t* offsets, int32_t* status, void* ws, void* const* ev,
+                 cudaStream_t st)
+{
+    const FwdLayout L = fwd_layout(c);
+    const bool shared = c.I_shared > 0;
+    float* lg = logits ? logits : at<float>(ws, L.logits);
+    int32_t* ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
+    float* w = topk_w ? topk_w : at<float>(ws, L.w);
+    int32_t* offs = offsets ? offsets : at<int32_t>(ws, L.offsets);
+    int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t* dest_row = at<int32_t>(ws, L.dest_row);
+    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+    uint16_t* y = at<uint16_t>(ws, L.y);
+    uint16_t* y_s = shared ? at<uint16_t>(ws, L.y_s) : nullptr;
+    int rc;
+    if ((rc = cuda_rc(router_logits(c, x, w_router, logit_bias, lg, status, st))) != MOE_OK)
+        return rc;
+    if ((rc = rec(ev, 1, st)) != MOE_OK) return rc;
+    if ((rc = cuda_rc(launch_route(c, lg, sel_bias, token_mask, ids, w, status, st))) != MOE_OK)
+        return rc;
+    if ((rc = rec(ev, 2, st)) != MOE_OK) return rc;
+    rc = cuda_rc(launch_permute(c, ids, offs, perm_token, dest_row, status,
+                                at<void>(ws, L.perm_ws), st));
+    if (rc != MOE_OK) return rc;
+    // materialised dispatch: the gather fused into the GEMM's operand loads is slower here
+    if ((rc = cuda_rc(launch_gather_rows(c, x, dest_row, x_perm, st))) != MOE_OK) return rc;
+    if ((rc = rec(ev, 3, st)) != MOE_OK) return rc;
+    rc = ffn_impl(c, x, x_perm, perm_token, offs, w13, w2, shared ? w13_s : nullptr,
+                  shared ? w2_s : nullptr, y, y_s, status, at<void>(ws, L.ffn), ev, st);
+    if (rc != MOE_OK) return rc;
+    rc = cuda_rc(launch_combine(c, y, w, dest_row, y_s, token_mask, out, st));
+    if (rc != MOE_OK) return rc;
+    return rec(ev, 7, st);
+}
+
+// scratch of moe_forward_host: the forward workspace of one chunk, then two x chunks and
+// two out chunks (double buffering)
+struct HostLayout {
+    int chunk;
+    size_t fwd, x_buf[2], out_buf[2], total;
+};
+
+HostLayout host_layout(const moe_cfg& c, int chunk_tokens)
+{
+    HostLayout L{};
+    L.chunk = chunk_tokens < c.T ? chunk_tokens : (c.T > 0 ? c.T : 1);
+    moe_cfg cc = c;
+    cc.T = L.chunk;
+    const size_t buf = up((size_t)L.chunk * c.H * 2);
+    size_t off = 0;
+    L.fwd = off;        off += fwd_layout(cc).total;
+    L.x_buf[0] = off;   off += buf;
+    L.x_buf[1] = off;   off += buf;
+    L.out_buf[0] = off; off += buf;
+    L.out_buf[1] = off; off += buf;
+    L.total = off;
+    return L;
+}
+
+// copy streams and events of moe_forward_host, created once per device and kept for the
+// life of the process (driver objects, no device memory)
+struct HostPipe {
+    cudaStream_t in, out;
+    cudaEvent_t start, done, copied_in[2], computed[2], copied_out[2];
+};
+
+cudaError_t host_pipe(HostPipe** out)
+{
+    static std::mutex mu;
+    static HostPipe* pipes[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (pipes[dev] == nullptr) {
+        HostPipe* p = new HostPipe();
+        if ((e = cudaStreamCreateWithFlags(&p->in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&p->out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        cudaEvent_t* evs[] = {&p->start, &p->done, &p->copied_in[0], &p->copied_in[1],
+                              &p->computed[0], &p->computed[1], &p->copied_out[0],
+                              &p->copied_out[1]};
+        for (cudaEvent_t* ev : evs)
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        pipes[dev] = p;
+    }
+    *out = pipes[dev];
+    return cudaSuccess;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -371,55 +486,88 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
                         float* topk_w, int32_t* offsets, int32_t* status, void* ws,
                         size_t ws_bytes, void* const* stage_events, void* stream)
 {
-    int rc = check_cfg(cfg);
+    int rc = check_forward_args(cfg, x, w_router, w13, w2, w13_s, w2_s, out, status);
     if (rc != MOE_OK) return rc;
+    const FwdLayout L = fwd_layout(*cfg);
+    if (ws == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (cfg->T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = rec(stage_events, 0, st)) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    return forward_impl(*cfg, x, w_router, logit_bias, sel_bias, token_mask, w13, w2, w13_s, w2_s,
+                        out, logits, topk_ids, topk_w, offsets, status, ws, stage_events, st);
+}
+
+MOE_API size_t moe_forward_host_workspace_bytes(const moe_cfg* cfg, int chunk_tokens)
+{
+    if (check_cfg(cfg) != MOE_OK || chunk_tokens < 1) return 0;
+    const HostLayout L = host_layout(*cfg, chunk_tokens);
+    return L.total;
+}
+
+MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const uint16_t* w_router,
+                             const float* logit_bias, const float* sel_bias,
+                             const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                             const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out_host,
+                             int32_t* status, int chunk_tokens, void* ws, size_t ws_bytes,
+                             void* stream)
+{
+    int rc = check_forward_args(cfg, x_host, w_router, w13, w2, w13_s, w2_s, out_host, status);
+    if (rc != MOE_OK) return rc;
+    if (chunk_tokens < 1) return MOE_ERR_ARG;
     const moe_cfg& c = *cfg;
-    if (x == nullptr || w_router == nullptr || w13 == nullptr || w2 == nullptr || out == nullptr ||
-        status == nullptr)
-        return MOE_ERR_ARG;
-    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) ||
-        !aligned16(out))
-        return MOE_ERR_ARG;
-    const bool shared = c.I_shared > 0;
-    if (shared && (w13_s == nullptr || w2_s == nullptr || !aligned16(w13_s) || !aligned16(w2_s)))
-        return MOE_ERR_ARG;
-    const FwdLayout L = fwd_layout(c);
+    const HostLayout L = host_layout(c, chunk_tokens);
     if (ws == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     if (c.T == 0) return MOE_OK;
     if ((rc = check_device()) != MOE_OK) return rc;
+    HostPipe* hp = nullptr;
+    if ((rc = cuda_rc(host_pipe(&hp))) != MOE_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    void* const* ev = stage_events;
-
-    float* lg = logits ? logits : at<float>(ws, L.logits);
-    int32_t* ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
-    float* w = topk_w ? topk_w : at<float>(ws, L.w);
-    int32_t* offs = offsets ? offsets : at<int32_t>(ws, L.offsets);
-    int32_t* perm_token = at<int32_t>(ws, L.perm_token);
-    int32_t* dest_row = at<int32_t>(ws, L.dest_row);
-    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
-    uint16_t* y = at<uint16_t>(ws, L.y);
-    uint16_t* y_s = shared ? at<uint16_t>(ws, L.y_s) : nullptr;
-
-    if ((rc = rec(ev, 0, st)) != MOE_OK) return rc;
+    const int C = L.chunk;
+    const size_t row_bytes = (size_t)c.H * 2;
     if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
-    if ((rc = cuda_rc(router_logits(c, x, w_router, logit_bias, lg, status, st))) != MOE_OK)
-        return rc;
-    if ((rc = rec(ev, 1, st)) != MOE_OK) return rc;
-    if ((rc = cuda_rc(launch_route(c, lg, sel_bias, token_mask, ids, w, status, st))) != MOE_OK)
-        return rc;
-    if ((rc = rec(ev, 2, st)) != MOE_OK) return rc;
-    rc = cuda_rc(launch_permute(c, ids, offs, perm_token, dest_row, status,
-                                at<void>(ws, L.perm_ws), st));
-    if (rc != MOE_OK) return rc;
-    // materialised dispatch: the gather fused into the GEMM's operand loads is slower here
-    if ((rc = cuda_rc(launch_gather_rows(c, x, dest_row, x_perm, st))) != MOE_OK) return rc;
-    if ((rc = rec(ev, 3, st)) != MOE_OK) return rc;
-    rc = ffn_impl(c, x, x_perm, perm_token, offs, w13, w2, shared ? w13_s : nullptr, shared ? w2_s : nullptr,
-                  y, y_s, status, at<void>(ws, L.ffn), ev, st);
-    if (rc != MOE_OK) return rc;
-    rc = cuda_rc(launch_combine(c, y, w, dest_row, y_s, token_mask, out, st));
-    if (rc != MOE_OK) return rc;
-    return rec(ev, 7, st);
+    // the copy streams start after everything already queued on the caller's stream
+    if ((rc = cuda_rc(cudaEventRecord(hp->start, st))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaStreamWaitEvent(hp->in, hp->start, 0))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaStreamWaitEvent(hp->out, hp->start, 0))) != MOE_OK) return rc;
+    const int n_chunks = (c.T + C - 1) / C;
+    for (int i = 0; i < n_chunks; ++i) {
+        const int slot = i & 1;
+        const int t0 = i * C;
+        const int tn = (c.T - t0) < C ? (c.T - t0) : C;
+        uint16_t* xb = at<uint16_t>(ws, L.x_buf[slot]);
+        uint16_t* ob = at<uint16_t>(ws, L.out_buf[slot]);
+        // H2D of chunk i once the compute of chunk i-2 no longer reads this x buffer
+        if (i >= 2 && (rc = cuda_rc(cudaStreamWaitEvent(hp->in, hp->computed[slot], 0))) != MOE_OK)
+            return rc;
+        rc = cuda_rc(cudaMemcpyAsync(xb, x_host + (size_t)t0 * c.H, (size_t)tn * row_bytes,
+                                     cudaMemcpyHostToDevice, hp->in));
+        if (rc != MOE_OK) return rc;
+        if ((rc = cuda_rc(cudaEventRecord(hp->copied_in[slot], hp->in))) != MOE_OK) return rc;
+        // compute of chunk i on the caller's stream, after its input landed and after the
+        // D2H of chunk i-2 has read this out buffer
+        if ((rc = cuda_rc(cudaStreamWaitEvent(st, hp->copied_in[slot], 0))) != MOE_OK) return rc;
+        if (i >= 2 && (rc = cuda_rc(cudaStreamWaitEvent(st, hp->copied_out[slot], 0))) != MOE_OK)
+            return rc;
+        moe_cfg cc = c;
+        cc.T = tn;
+        rc = forward_impl(cc, xb, w_router, logit_bias, sel_bias,
+                          token_mask ? token_mask + t0 : nullptr, w13, w2, w13_s, w2_s, ob,
+                          nullptr, nullptr, nullptr, nullptr, status, at<void>(ws, L.fwd),
+                          nullptr, st);
+        if (rc != MOE_OK) return rc;
+        if ((rc = cuda_rc(cudaEventRecord(hp->computed[slot], st))) != MOE_OK) return rc;
+        // D2H of chunk i
+        if ((rc = cuda_rc(cudaStreamWaitEvent(hp->out, hp->computed[slot], 0))) != MOE_OK) return rc;
+        rc = cuda_rc(cudaMemcpyAsync(out_host + (size_t)t0 * c.H, ob, (size_t)tn * row_bytes,
+                                     cudaMemcpyDeviceToHost, hp->out));
+        if (rc != MOE_OK) return rc;
+        if ((rc = cuda_rc(cudaEventRecord(hp->copied_out[slot], hp->out))) != MOE_OK) return rc;
+    }
+    // the caller's stream completes only after the last result reached the host
+    if ((rc = cuda_rc(cudaEventRecord(hp->done, hp->out))) != MOE_OK) return rc;
+    return cuda_rc(cudaStreamWaitEvent(st, hp->done, 0));
 }
 
 }  // extern "C"

@@ -264,6 +264,43 @@ def forward(cfg: Config, x, w_router, w13, w2, logit_bias=None, sel_bias=None, t
     return (out, b) if keep else out
 
 
+def forward_host_workspace_bytes(cfg: Config, chunk: int) -> int:
+    return int(N.load().moe_forward_host_workspace_bytes(ctypes.byref(cfg.c()), int(chunk)))
+
+
+def forward_host(cfg: Config, x_host, w_router, w13, w2, logit_bias=None, sel_bias=None,
+                 token_mask=None, w13_s=None, w2_s=None, out_host=None, chunk: int = 4096,
+                 ws=None, status=None, check: bool = True):
+    """The layer from and to host memory in one C-ABI call, transfers overlapped with the
+    compute in chunks of `chunk` tokens. x_host / out_host are CPU bf16 tensors (pin them
+    for the overlap); weights, biases and the mask are on the device."""
+    dev = w13.device
+    T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
+    cpu = torch.device("cpu")
+    _need(x_host, "x_host", torch.bfloat16, (T, H), cpu)
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory() if out_host is None \
+        else out_host
+    _need(out_host, "out_host", torch.bfloat16, (T, H), cpu)
+    _need(w_router, "w_router", torch.bfloat16, (E, H), dev)
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H), dev)
+    _need(w2, "w2", torch.bfloat16, (E, H, I), dev)
+    _opt(logit_bias, "logit_bias", torch.float32, (E,), dev)
+    _opt(sel_bias, "sel_bias", torch.float32, (E,), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    if Is:
+        _need(w13_s, "w13_s", torch.bfloat16, (2 * Is, H), dev)
+        _need(w2_s, "w2_s", torch.bfloat16, (H, Is), dev)
+    ws = _ws(forward_host_workspace_bytes(cfg, chunk), dev, ws)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_forward_host(ctypes.byref(cfg.c()), _p(x_host), _p(w_router),
+                                  _p(logit_bias), _p(sel_bias), _p(token_mask), _p(w13), _p(w2),
+                                  _p(w13_s), _p(w2_s), _p(out_host), _p(st), int(chunk), _p(ws),
+                                  ws.numel(), _stream(dev)), "moe_forward_host")
+    if check:
+        check_status(st)
+    return out_host
+
+
 class MoELayer:
     """A layer holding its weights and a reusable workspace sized for up to max_T tokens.
 
@@ -277,6 +314,20 @@ class MoELayer:
         dev = weights["w13"].device
         self.ws = _ws(workspace_bytes(cfg.with_T(self.max_T), N.MOE_STAGE_FORWARD), dev, None)
         self.status = new_status(dev)
+
+    def forward_host(self, x_host, out_host=None, chunk: int = 4096, token_mask=None,
+                     check=True):
+        """The layer from pinned host memory to pinned host memory (see forward_host)."""
+        T = x_host.shape[0]
+        need = forward_host_workspace_bytes(self.cfg.with_T(T), chunk)
+        if getattr(self, "_host_ws", None) is None or self._host_ws.numel() < need:
+            self._host_ws = _ws(need, self.ws.device, None)
+        w = self.w
+        return forward_host(self.cfg.with_T(T), x_host, w["w_router"], w["w13"], w["w2"],
+                            logit_bias=w.get("logit_bias"), sel_bias=w.get("sel_bias"),
+                            token_mask=token_mask, w13_s=w.get("w13_s"), w2_s=w.get("w2_s"),
+                            out_host=out_host, chunk=chunk, ws=self._host_ws,
+                            status=self.status, check=check)
 
     def __call__(self, x, token_mask=None, out=None, keep=False, check=True, stage_events=None):
         T = x.shape[0]

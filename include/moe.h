@@ -239,6 +239,30 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
                         int32_t* status, void* ws, size_t ws_bytes, void* const* stage_events,
                         void* stream);
 
+/*
+ * The whole layer from and to HOST memory, overlapping the transfers with the compute
+ * (the chunked form is exact: results are bitwise independent of how tokens are split).
+ * Tokens are processed in chunks of `chunk_tokens`: the host->device copy of chunk i+1 and
+ * the device->host copy of chunk i-1 run on two library-owned copy streams while chunk i
+ * runs on `stream`, double-buffered in `ws`. When `stream` completes, out_host holds the
+ * result. Same output bits as moe_forward on the same tokens.
+ *
+ *  x_host       [T,H] bf16 in HOST memory (page-locked for the copies to overlap).
+ *  out_host     [T,H] bf16 in HOST memory (page-locked).
+ *  token_mask   [T] uint8 in DEVICE memory, or NULL.
+ *  weights, biases, status: DEVICE, as in moe_forward.
+ *  ws           moe_forward_host_workspace_bytes(cfg, chunk_tokens) bytes (device).
+ * The copy streams and their events are created on a device's first call and kept until
+ * the process exits; calls on one device must not overlap in host threads.
+ */
+MOE_API size_t moe_forward_host_workspace_bytes(const moe_cfg* cfg, int chunk_tokens);
+MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const uint16_t* w_router,
+                             const float* logit_bias, const float* sel_bias,
+                             const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                             const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out_host,
+                             int32_t* status, int chunk_tokens, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Text of a return code. */
 MOE_API const char* moe_status_string(int code);
 

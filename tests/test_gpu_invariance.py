@@ -139,3 +139,22 @@ def test_sigmoid_shared_expert_layer_invariance():
     mask = torch.zeros(T, dtype=torch.uint8, device=DEV)
     mask[17:17 + sw.n] = 1
     same(sw.pick(sw.run(x, mask), np.arange(17, 17 + sw.n)), ref, "masked padding")
+
+
+@pytest.mark.parametrize("name,T,chunks", [("qwen3_30b_a3b", 4096, (1000, 2048, 4096, 8192)),
+                                           ("tiny", 333, (7, 64, 333)),
+                                           ("dsv_sigmoid", 1500, (512,))])
+def test_forward_host_chunked_equals_forward(name, T, chunks):
+    """The host-memory entry point (chunked, copies overlapped) gives the bits of one
+    moe_forward on device memory, for any chunk size, with and without a mask."""
+    s, d = synthetic.make_layer(name, T=T, device=DEV)
+    cfg = moe.Config.of(s)
+    mask = synthetic.random_mask(T, 0.85, 3).to(DEV)
+    w = dict(logit_bias=d["logit_bias"], sel_bias=d["sel_bias"], w13_s=d["w13_s"], w2_s=d["w2_s"])
+    x_host = d["x"].cpu().pin_memory()
+    for m in (None, mask):
+        ref = moe.forward(cfg, d["x"], d["w_router"], d["w13"], d["w2"], token_mask=m, **w)
+        for c in chunks:
+            out = moe.forward_host(cfg, x_host, d["w_router"], d["w13"], d["w2"], token_mask=m,
+                                   chunk=c, **w)
+            assert np.array_equal(bits(out), bits(ref)), (name, c, m is not None)
