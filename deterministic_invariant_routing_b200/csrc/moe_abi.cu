@@ -119,27 +119,27 @@ int rec(void* const* ev, int i, cudaStream_t st)
     return cuda_rc(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st));
 }
 
-// router logits on the tensor cores: logits[T,E] = x . Wr^T (+ bias), fp32
-cudaError_t router_logits(const moe_cfg& c, const uint16_t* x, const uint16_t* wr,
-                          const float* logit_bias, float* logits, int32_t* status,
-                          cudaStream_t st)
+// router on the tensor cores (logits[T,E] = x . Wr^T + bias, fp32), then the routing kernel
+int router_and_route(const moe_cfg& c, const uint16_t* x, const uint16_t* wr,
+                     const float* logit_bias, const float* sel_bias, const uint8_t* mask,
+                     float* logits, int32_t* ids, float* w, int32_t* status, void* const* ev,
+                     cudaStream_t st)
 {
-    GemmProblem p{};
-    p.epilogue = EPI_F32;
-    p.a = x;
-    p.a_rows = c.T;
-    p.b = wr;
-    p.b_rows_per_group = c.E;
-    p.k = c.H;
-    p.n = c.E;
-    p.groups = 1;
-    p.offsets = nullptr;
-    p.rows = c.T;
-    p.out = logits;
-    p.ldo = c.E;
-    p.bias = logit_bias;
+    RouterProblem p{};
+    p.x = x;
+    p.w_router = wr;
+    p.T = c.T;
+    p.H = c.H;
+    p.E = c.E;
+    p.logit_bias = logit_bias;
+    p.logits = logits;
     p.status = status;
-    return launch_tc_gemm(p, st);
+    int rc;
+    if ((rc = cuda_rc(launch_router(p, st))) != MOE_OK) return rc;
+    if ((rc = rec(ev, 1, st)) != MOE_OK) return rc;
+    if ((rc = cuda_rc(launch_route(c, logits, sel_bias, mask, ids, w, status, st))) != MOE_OK)
+        return rc;
+    return rec(ev, 2, st);
 }
 
 // gate_up + SwiGLU over grouped rows: h[r] = silu(a_r . W1g^T) * (a_r . W1u^T), where
@@ -165,7 +165,7 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
     p.out = h;
     p.ldo = I;
     p.status = status;
-    return launch_tc_gemm(p, st);
+    return launch_tc_gemm_pair(p, st);
 }
 
 // down over grouped rows: y[r] = h_r . W2^T
@@ -187,7 +187,7 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     p.out = y;
     p.ldo = H;
     p.status = status;
-    return launch_tc_gemm(p, st);
+    return launch_tc_gemm_pair(p, st);
 }
 
 int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm,
@@ -257,13 +257,9 @@ int forward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* w_router,
     uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
     uint16_t* y = at<uint16_t>(ws, L.y);
     uint16_t* y_s = shared ? at<uint16_t>(ws, L.y_s) : nullptr;
-    int rc;
-    if ((rc = cuda_rc(router_logits(c, x, w_router, logit_bias, lg, status, st))) != MOE_OK)
-        return rc;
-    if ((rc = rec(ev, 1, st)) != MOE_OK) return rc;
-    if ((rc = cuda_rc(launch_route(c, lg, sel_bias, token_mask, ids, w, status, st))) != MOE_OK)
-        return rc;
-    if ((rc = rec(ev, 2, st)) != MOE_OK) return rc;
+    int rc = router_and_route(c, x, w_router, logit_bias, sel_bias, token_mask, lg, ids, w,
+                              status, ev, st);
+    if (rc != MOE_OK) return rc;
     rc = cuda_rc(launch_permute(c, ids, offs, perm_token, dest_row, status,
                                 at<void>(ws, L.perm_ws), st));
     if (rc != MOE_OK) return rc;
@@ -384,10 +380,9 @@ MOE_API int moe_route(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_r
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (status && (rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK)
         return rc;
-    if (x != nullptr) {
-        rc = cuda_rc(router_logits(*cfg, x, w_router, logit_bias, logits, status, st));
-        if (rc != MOE_OK) return rc;
-    }
+    if (x != nullptr)
+        return router_and_route(*cfg, x, w_router, logit_bias, sel_bias, token_mask, logits,
+                                topk_ids, topk_w, status, nullptr, st);
     return cuda_rc(launch_route(*cfg, logits, sel_bias, token_mask, topk_ids, topk_w, status, st));
 }
 

@@ -41,7 +41,7 @@ cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
                            const uint8_t* mask, uint16_t* out, cudaStream_t st);
 
 // tensor-core GEMMs (tcgen05 / TMEM / TMA)
-enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_F32 = 2 };
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1 };
 
 struct GemmProblem {
     int epilogue;            // GemmEpilogue
@@ -62,8 +62,19 @@ struct GemmProblem {
     int32_t* status;         // device status words (MOE_ST_PIPE_TIMEOUT) or NULL
 };
 
-cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st);
+// the grouped expert products (EPI_SWIGLU / EPI_BF16) on CTA pairs
 cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st);
+
+// the router product: logits[T,E] = x . Wr^T (+ logit_bias), fp32
+struct RouterProblem {
+    const uint16_t* x;         // [T,H] bf16
+    const uint16_t* w_router;  // [E,H] bf16
+    int T, H, E;
+    const float* logit_bias;   // [E] or NULL
+    float* logits;             // [T,E] fp32 out
+    int32_t* status;
+};
+cudaError_t launch_router(const RouterProblem& p, cudaStream_t st);
 
 // device facts
 int num_sms();

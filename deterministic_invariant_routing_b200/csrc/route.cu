@@ -10,50 +10,10 @@
 // the softmax denominator is the 32-lane tree (lane L sums experts L, L+32, ... in
 // increasing order, then butterfly levels 16, 8, 4, 2, 1); the selection compares
 // 64-bit keys (ordered choice bits, then inverted id), so ties go to the lower id.
-#include "moe_internal.cuh"
+#include "route_math.cuh"
 
 namespace moe {
 namespace {
-
-// exp_rl: Cody & Waite additive range reduction (x = n ln2 + r, ln2 split in a 12-bit
-// head whose products with n are exact and an fp32 tail), then the degree-7 Taylor
-// polynomial of e^r by Horner with fused multiply-adds, scaled by 2^n built from the
-// exponent field. Specials: NaN -> NaN, x < -87 -> +0, x > 88 -> +inf.
-__device__ __forceinline__ float exp_rl(float x)
-{
-    // ln 2 rounded to the nearest multiple of 2^-12 (12 significant bits: n * head is
-    // exact for |n| <= 127), and the fp32 rounding of the remainder.
-    const double kLn2 = 0.693147180559945309417232121458;
-    const float kHead = __double2float_rn(rint(kLn2 * 4096.0) / 4096.0);
-    const float kTail = __double2float_rn(kLn2 - (double)kHead);
-    const float kLog2e = __double2float_rn(1.442695040888963407359924681002);
-    if (isnan(x)) return x;
-    if (x < -87.0f) return 0.0f;
-    if (x > 88.0f) return __int_as_float(0x7f800000);
-    const float n = rintf(__fmul_rn(x, kLog2e));
-    float r = __fmaf_rn(-n, kHead, x);
-    r = __fmaf_rn(-n, kTail, r);
-    // Taylor coefficients 1/k!, k = 7 .. 0, each rounded once to fp32
-    float p = __double2float_rn(1.0 / 5040.0);
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 720.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 120.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 24.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 6.0));
-    p = __fmaf_rn(p, r, 0.5f);
-    p = __fmaf_rn(p, r, 1.0f);
-    p = __fmaf_rn(p, r, 1.0f);
-    const float two_n = __int_as_float((__float2int_rn(n) + 127) << 23);
-    return __fmul_rn(p, two_n);
-}
-
-// order-preserving 32-bit image of a choice: -0 == +0, NaN below every number
-__device__ __forceinline__ uint32_t order_bits(float c)
-{
-    if (isnan(c)) return 0u;
-    if (c == 0.0f) c = 0.0f;
-    const uint32_t u = __float_as_uint(c);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b)
 {
@@ -139,10 +99,12 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             unsigned long long best = 0ull;
 #pragma unroll
             for (int i = 0; i < NE; ++i) best = umax64(best, key[i]);
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                best = umax64(best, __shfl_xor_sync(0xffffffffu, best, off));
-            const int e = (int)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
+            // warp arg-max of the 64-bit keys as two 32-bit reductions: the highest choice
+            // bits, then, among the lanes holding them, the highest inverted id
+            const uint32_t hi = (uint32_t)(best >> 32), lo = (uint32_t)best;
+            const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+            const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+            const int e = (int)(0xffffffffu - mlo);
             const int owner = e & 31, slot = e >> 5;
             float se = 0.0f;
 #pragma unroll
