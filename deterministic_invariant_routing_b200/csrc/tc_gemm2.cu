@@ -437,6 +437,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (err != cudaSuccess) return err;
     static bool attr_set[64] = {};
     static int max_clusters[64] = {};
+    static size_t max_smem[64] = {};
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -452,14 +453,17 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (!attr_set[dev]) {
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
         if (err != cudaSuccess) return err;
+        attr_set[dev] = true;
+    }
+    if (max_clusters[dev] == 0 || smem > max_smem[dev]) {
+        // co-resident clusters at this shared-memory size (one CTA per SM in practice)
         cfg.gridDim = dim3(2 * 74, 1, 1);
-        cfg.dynamicSmemBytes = C::smem_bytes(1025);
         int n = 0;
         err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
         if (err != cudaSuccess) return err;
-        max_clusters[dev] = n > 0 ? n : 1;
-        cfg.dynamicSmemBytes = smem;
-        attr_set[dev] = true;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        max_clusters[dev] = n;
+        max_smem[dev] = smem;
     }
     CUtensorMap ma, mb;
     if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) return cudaErrorInvalidValue;
