@@ -112,6 +112,105 @@ cudaError_t launch_k(const moe_cfg& c, const uint16_t* y, const float* w, const 
     return cudaGetLastError();
 }
 
+// Order-invariant variant ("From Expert Reduction to Behavioral Divergence", arXiv
+// 2607.28097, Abstract: scheme C's result does not depend on the order of the expert
+// terms). Per output element the terms -- w_j * y_j formed exactly in double, and the
+// shared expert's y -- are put in a canonical order (ascending magnitude, the negative of
+// equal magnitudes first) by an odd-even transposition network, summed in double, and
+// rounded once to fp32 then to bf16. The result is a function of the multiset of terms.
+__device__ __forceinline__ bool canon_after(double a, bool va, double b, bool vb)
+{
+    // should slot a (valid va) come after slot b? invalid slots go last
+    if (!va) return vb;
+    if (!vb) return false;
+    const double fa = fabs(a), fb = fabs(b);
+    return fa != fb ? fa > fb : a > b;
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(256) combine_invariant_kernel(
+    const uint4* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ dest_row,
+    const uint4* __restrict__ y_shared, const uint8_t* __restrict__ mask, int T, int K,
+    int vec_per_row, uint4* __restrict__ out)
+{
+    constexpr int N = KMAX + 1;
+    const int64_t total = (int64_t)T * vec_per_row;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = idx / vec_per_row;
+        const int v = (int)(idx - t * vec_per_row);
+        if (mask != nullptr && mask[t] == 0) {
+            out[idx] = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        uint4 rows[N];
+        float wj[N];
+        bool ok[N];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            const int32_t r = (j < K) ? dest_row[t * K + j] : -1;
+            ok[j] = r >= 0;
+            wj[j] = ok[j] ? w[t * K + j] : 0.0f;
+            rows[j] = ok[j] ? y[(int64_t)r * vec_per_row + v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+        ok[KMAX] = y_shared != nullptr;
+        wj[KMAX] = 1.0f;
+        rows[KMAX] = ok[KMAX] ? y_shared[idx] : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t packed[4];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            double term[N];
+            bool val[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                const uint32_t q = (c >> 1) == 0 ? rows[j].x
+                                 : (c >> 1) == 1 ? rows[j].y
+                                 : (c >> 1) == 2 ? rows[j].z : rows[j].w;
+                const float yv = (c & 1) ? bf16_hi(q) : bf16_lo(q);
+                term[j] = __dmul_rn((double)wj[j], (double)yv);  // exact
+                val[j] = ok[j];
+            }
+#pragma unroll
+            for (int pass = 0; pass < N; ++pass) {
+#pragma unroll
+                for (int i = pass & 1; i + 1 < N; i += 2) {
+                    if (canon_after(term[i], val[i], term[i + 1], val[i + 1])) {
+                        const double td = term[i];
+                        term[i] = term[i + 1];
+                        term[i + 1] = td;
+                        const bool tv = val[i];
+                        val[i] = val[i + 1];
+                        val[i + 1] = tv;
+                    }
+                }
+            }
+            double sum = 0.0;
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+                if (val[j]) sum = __dadd_rn(sum, term[j]);
+            const float f = __double2float_rn(sum);
+            if (c & 1) packed[c >> 1] |= pack_bf16(0.0f, f) & 0xffff0000u;
+            else packed[c >> 1] = pack_bf16(f, 0.0f) & 0xffffu;
+        }
+        out[idx] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
+template <int KMAX>
+cudaError_t launch_inv(const moe_cfg& c, const uint16_t* y, const float* w, const int32_t* dr,
+                       const uint16_t* ys, const uint8_t* mask, uint16_t* out, cudaStream_t st)
+{
+    const int vec = c.H / 8;
+    const int64_t total = (int64_t)c.T * vec;
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    combine_invariant_kernel<KMAX><<<(unsigned)blocks, 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys), mask,
+        c.T, c.K, vec, reinterpret_cast<uint4*>(out));
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
@@ -124,6 +223,17 @@ cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
     if (c.K <= 4) return launch_k<4>(c, y, w, dest_row, y_shared, mask, out, st);
     if (c.K <= 8) return launch_k<8>(c, y, w, dest_row, y_shared, mask, out, st);
     return launch_k<16>(c, y, w, dest_row, y_shared, mask, out, st);
+}
+
+cudaError_t launch_combine_invariant(const moe_cfg& c, const uint16_t* y, const float* w,
+                                     const int32_t* dest_row, const uint16_t* y_shared,
+                                     const uint8_t* mask, uint16_t* out, cudaStream_t st)
+{
+    if (c.T == 0) return cudaSuccess;
+    if (c.K <= 2) return launch_inv<2>(c, y, w, dest_row, y_shared, mask, out, st);
+    if (c.K <= 4) return launch_inv<4>(c, y, w, dest_row, y_shared, mask, out, st);
+    if (c.K <= 8) return launch_inv<8>(c, y, w, dest_row, y_shared, mask, out, st);
+    return launch_inv<16>(c, y, w, dest_row, y_shared, mask, out, st);
 }
 
 }  // namespace moe

@@ -361,6 +361,7 @@ MOE_API size_t moe_workspace_bytes(const moe_cfg* cfg, int stage)
         case MOE_STAGE_FFN: return ffn_layout(*cfg).total;
         case MOE_STAGE_COMBINE: return 0;
         case MOE_STAGE_FORWARD: return fwd_layout(*cfg).total;
+        case MOE_STAGE_STATS: return stats_ws_bytes(*cfg);
         default: return 0;
     }
 }
@@ -474,6 +475,22 @@ MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* y, const float* topk
                                   static_cast<cudaStream_t>(stream)));
 }
 
+MOE_API int moe_combine_invariant(const moe_cfg* cfg, const uint16_t* y, const float* topk_w,
+                                  const int32_t* dest_row, const uint16_t* y_shared,
+                                  const uint8_t* token_mask, uint16_t* out, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (y == nullptr || topk_w == nullptr || dest_row == nullptr || out == nullptr)
+        return MOE_ERR_ARG;
+    if (!aligned16(y) || !aligned16(out) || (y_shared != nullptr && !aligned16(y_shared)))
+        return MOE_ERR_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    return cuda_rc(launch_combine_invariant(*cfg, y, topk_w, dest_row, y_shared, token_mask, out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
                         const float* logit_bias, const float* sel_bias, const uint8_t* token_mask,
                         const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s,
@@ -492,6 +509,22 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
     if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
     return forward_impl(*cfg, x, w_router, logit_bias, sel_bias, token_mask, w13, w2, w13_s, w2_s,
                         out, logits, topk_ids, topk_w, offsets, status, ws, stage_events, st);
+}
+
+MOE_API int moe_router_stats(const moe_cfg* cfg, const float* logits, const uint8_t* token_mask,
+                             const int32_t* offsets, int32_t* tokens_per_expert,
+                             float* mean_prob, float* aux, void* ws, size_t ws_bytes,
+                             void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    if (logits == nullptr || offsets == nullptr || tokens_per_expert == nullptr ||
+        mean_prob == nullptr || aux == nullptr)
+        return MOE_ERR_ARG;
+    if (ws == nullptr || ws_bytes < stats_ws_bytes(*cfg)) return MOE_ERR_WORKSPACE;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    return cuda_rc(launch_router_stats(*cfg, logits, token_mask, offsets, tokens_per_expert,
+                                       mean_prob, aux, ws, static_cast<cudaStream_t>(stream)));
 }
 
 MOE_API size_t moe_forward_host_workspace_bytes(const moe_cfg* cfg, int chunk_tokens)

@@ -35,10 +35,21 @@ cudaError_t permute_fixed_scratch(int32_t** out);
 cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_t* dest_row,
                                uint16_t* x_perm, cudaStream_t st);
 
+// router statistics (tokens per expert, mean L1-normalised score, load-balance value)
+size_t stats_ws_bytes(const moe_cfg& c);
+cudaError_t launch_router_stats(const moe_cfg& c, const float* logits, const uint8_t* mask,
+                                const int32_t* offsets, int32_t* counts, float* mean_prob,
+                                float* aux, void* ws, cudaStream_t st);
+
 // combine
 cudaError_t launch_combine(const moe_cfg& c, const uint16_t* y, const float* w,
                            const int32_t* dest_row, const uint16_t* y_shared,
                            const uint8_t* mask, uint16_t* out, cudaStream_t st);
+
+// order-invariant combine (canonical-order double sum of the exact terms)
+cudaError_t launch_combine_invariant(const moe_cfg& c, const uint16_t* y, const float* w,
+                                     const int32_t* dest_row, const uint16_t* y_shared,
+                                     const uint8_t* mask, uint16_t* out, cudaStream_t st);
 
 // tensor-core GEMMs (tcgen05 / TMEM / TMA)
 enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1 };

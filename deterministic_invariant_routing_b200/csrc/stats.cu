@@ -1,0 +1,193 @@
+// Router statistics of one routed batch (SpecForge PR #1003, the load-balance commit): the
+// tokens per expert, the mean L1-normalised score per expert and the Switch-style
+// load-balance value  aux = E * sum_e load_e * mean_prob_e  over the kept tokens (K when
+// balanced), where load_e = tokens_per_expert_e / N and p_{t,e} = s_{t,e} / sum_e' s_{t,e'}
+// with s the unbiased scores of the routing contract (softmax or sigmoid).
+//
+// Deterministic without float atomics: block b owns 256 consecutive tokens, warp w of it
+// 32 of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
+// ...); the 8 warp partials are added in warp order, then the block partials in block order
+// by the finishing kernel, and aux is a fixed tree over the experts. The result depends on
+// T (a batch statistic), never on scheduling.
+#include "route_math.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTokPerBlock = 256;
+constexpr int kWarps = 8;
+constexpr int kTokPerWarp = kTokPerBlock / kWarps;
+
+template <int NE>
+__global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __restrict__ logits,
+                                                               const uint8_t* __restrict__ mask,
+                                                               int T, int E, int score_fn,
+                                                               float* __restrict__ partial,
+                                                               int32_t* __restrict__ kept)
+{
+    extern __shared__ float wsum[];  // [kWarps][E]
+    __shared__ int32_t wkept[kWarps];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    float acc[NE];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) acc[i] = 0.0f;
+    int n_kept = 0;
+    const int64_t t0 = (int64_t)blockIdx.x * kTokPerBlock + (int64_t)wid * kTokPerWarp;
+    for (int r = 0; r < kTokPerWarp; ++r) {
+        const int64_t t = t0 + r;
+        if (t >= T) break;
+        if (mask != nullptr && mask[t] == 0) continue;
+        ++n_kept;
+        const float* row = logits + t * E;
+        float s[NE];
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            s[i] = (e < E) ? row[e] : 0.0f;
+        }
+        if (score_fn == MOE_SIGMOID) {
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                if (lane + 32 * i < E) s[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_rl(-s[i])));
+        } else {
+            float m = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                if (lane + 32 * i < E && s[i] > m) m = s[i];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const float o = __shfl_xor_sync(0xffffffffu, m, off);
+                if (o > m) m = o;
+            }
+            float part = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                if (lane + 32 * i < E) {
+                    s[i] = exp_rl(__fsub_rn(s[i], m));
+                    part = __fadd_rn(part, s[i]);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
+#pragma unroll
+            for (int i = 0; i < NE; ++i) s[i] = __fdiv_rn(s[i], part);
+        }
+        // L1 normalisation over the experts with the same 32-lane tree
+        float l1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (lane + 32 * i < E) l1 = __fadd_rn(l1, s[i]);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+            l1 = __fadd_rn(l1, __shfl_xor_sync(0xffffffffu, l1, off));
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (lane + 32 * i < E) acc[i] = __fadd_rn(acc[i], __fdiv_rn(s[i], l1));
+    }
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) wsum[wid * E + e] = acc[i];
+    }
+    if (lane == 0) wkept[wid] = n_kept;
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float v = wsum[e];
+        for (int w = 1; w < kWarps; ++w) v = __fadd_rn(v, wsum[w * E + e]);
+        partial[(int64_t)blockIdx.x * E + e] = v;
+    }
+    if (threadIdx.x == 0) {
+        int k = 0;
+        for (int w = 0; w < kWarps; ++w) k += wkept[w];
+        kept[blockIdx.x] = k;
+    }
+}
+
+// one block of 1024 threads, thread e owns expert e
+__global__ void __launch_bounds__(1024) stats_finish_kernel(const float* __restrict__ partial,
+                                                            const int32_t* __restrict__ kept,
+                                                            int nblocks, int E,
+                                                            const int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ counts,
+                                                            float* __restrict__ mean_prob,
+                                                            float* __restrict__ aux)
+{
+    __shared__ float wsum[32];
+    const int e = threadIdx.x, lane = e & 31, wid = e >> 5;
+    int64_t n = 0;
+    for (int b = 0; b < nblocks; ++b) n += kept[b];
+    float term = 0.0f;
+    if (e < E) {
+        float v = 0.0f;
+        for (int b = 0; b < nblocks; ++b) v = __fadd_rn(v, partial[(int64_t)b * E + e]);
+        const int32_t c = offsets[e + 1] - offsets[e];
+        counts[e] = c;
+        const float nf = (float)n;
+        const float mp = n > 0 ? __fdiv_rn(v, nf) : 0.0f;
+        mean_prob[e] = mp;
+        term = n > 0 ? __fmul_rn(__fdiv_rn((float)c, nf), mp) : 0.0f;
+    }
+    // fixed tree over the experts: warp butterfly, then the 32 warp sums in order
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        term = __fadd_rn(term, __shfl_xor_sync(0xffffffffu, term, off));
+    if (lane == 0) wsum[wid] = term;
+    __syncthreads();
+    if (e == 0) {
+        float s = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s = __fadd_rn(s, wsum[w]);
+        *aux = __fmul_rn((float)E, s);
+    }
+}
+
+template <int NE>
+cudaError_t launch_ne(const moe_cfg& c, const float* logits, const uint8_t* mask, float* partial,
+                      int32_t* kept, int nb, cudaStream_t st)
+{
+    const size_t smem = (size_t)kWarps * c.E * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(prob_sum_kernel<NE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    prob_sum_kernel<NE><<<nb, kWarps * 32, smem, st>>>(logits, mask, c.T, c.E, c.score_fn,
+                                                       partial, kept);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t stats_ws_bytes(const moe_cfg& c)
+{
+    const int64_t nb = ((int64_t)c.T + kTokPerBlock - 1) / kTokPerBlock;
+    const int64_t n = nb > 0 ? nb : 1;
+    return (size_t)n * c.E * sizeof(float) + (size_t)n * sizeof(int32_t) + 256;
+}
+
+cudaError_t launch_router_stats(const moe_cfg& c, const float* logits, const uint8_t* mask,
+                                const int32_t* offsets, int32_t* counts, float* mean_prob,
+                                float* aux, void* ws, cudaStream_t st)
+{
+    const int nb = (int)(((int64_t)c.T + kTokPerBlock - 1) / kTokPerBlock);
+    float* partial = static_cast<float*>(ws);
+    int32_t* kept = reinterpret_cast<int32_t*>(
+        static_cast<char*>(ws) + (size_t)(nb > 0 ? nb : 1) * c.E * sizeof(float));
+    cudaError_t err = cudaSuccess;
+    if (nb > 0) {
+        const int ne = (c.E + 31) / 32;
+        if (ne <= 1) err = launch_ne<1>(c, logits, mask, partial, kept, nb, st);
+        else if (ne <= 2) err = launch_ne<2>(c, logits, mask, partial, kept, nb, st);
+        else if (ne <= 4) err = launch_ne<4>(c, logits, mask, partial, kept, nb, st);
+        else if (ne <= 8) err = launch_ne<8>(c, logits, mask, partial, kept, nb, st);
+        else if (ne <= 16) err = launch_ne<16>(c, logits, mask, partial, kept, nb, st);
+        else err = launch_ne<32>(c, logits, mask, partial, kept, nb, st);
+        if (err != cudaSuccess) return err;
+    }
+    stats_finish_kernel<<<1, 1024, 0, st>>>(partial, kept, nb, c.E, offsets, counts, mean_prob,
+                                            aux);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -196,8 +196,10 @@ def grouped_ffn(cfg: Config, x, x_perm, perm_token, offsets, w13, w2, w13_s=None
     return y, y_s
 
 
-def combine(cfg: Config, y, topk_w, dest_row, y_shared=None, token_mask=None):
-    """Reduction boundary. Returns out [T,H] bf16."""
+def combine(cfg: Config, y, topk_w, dest_row, y_shared=None, token_mask=None,
+            order_invariant: bool = False):
+    """Reduction boundary. Returns out [T,H] bf16. order_invariant=True runs the
+    canonical-order variant (moe_combine_invariant) instead of the rank-order contract."""
     dev = y.device
     T, H, K = cfg.T, cfg.H, cfg.K
     if y.dim() != 2 or y.shape[1] != H or y.dtype != torch.bfloat16 or not y.is_contiguous():
@@ -207,9 +209,29 @@ def combine(cfg: Config, y, topk_w, dest_row, y_shared=None, token_mask=None):
     _opt(y_shared, "y_shared", torch.bfloat16, (T, H), dev)
     _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    _rc(N.load().moe_combine(ctypes.byref(cfg.c()), _p(y), _p(topk_w), _p(dest_row),
-                             _p(y_shared), _p(token_mask), _p(out), _stream(dev)), "moe_combine")
+    fn = N.load().moe_combine_invariant if order_invariant else N.load().moe_combine
+    _rc(fn(ctypes.byref(cfg.c()), _p(y), _p(topk_w), _p(dest_row), _p(y_shared),
+           _p(token_mask), _p(out), _stream(dev)), "moe_combine")
     return out
+
+
+def router_stats(cfg: Config, logits, offsets, token_mask=None):
+    """Router statistics of a routed batch: {tokens_per_expert [E] int32, mean_prob [E]
+    fp32, aux [1] fp32} (the load-balance value E * sum_e load_e * mean_prob_e, K when
+    balanced). logits and offsets as returned by route()/permute() or forward(keep=True)."""
+    dev = logits.device
+    T, E = cfg.T, cfg.E
+    _need(logits, "logits", torch.float32, (T, E), dev)
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    mp = torch.empty(E, dtype=torch.float32, device=dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = _ws(workspace_bytes(cfg, N.MOE_STAGE_STATS), dev, None)
+    _rc(N.load().moe_router_stats(ctypes.byref(cfg.c()), _p(logits), _p(token_mask),
+                                  _p(offsets), _p(counts), _p(mp), _p(aux), _p(ws), ws.numel(),
+                                  _stream(dev)), "moe_router_stats")
+    return {"tokens_per_expert": counts, "mean_prob": mp, "aux": aux}
 
 
 # ------------------------------------------------------------------ whole layer

@@ -79,6 +79,7 @@ extern "C" {
 #define MOE_STAGE_FFN 2
 #define MOE_STAGE_COMBINE 3
 #define MOE_STAGE_FORWARD 4
+#define MOE_STAGE_STATS 5
 
 /* number of CUDA events moe_forward can record (stage boundaries), see moe_forward */
 #define MOE_NUM_STAGE_EVENTS 8
@@ -217,6 +218,20 @@ MOE_API int moe_combine(const moe_cfg* cfg, const uint16_t* y, const float* topk
                         const uint8_t* token_mask, uint16_t* out, void* stream);
 
 /*
+ * Order-invariant combine ("From Expert Reduction to Behavioral Divergence", arXiv
+ * 2607.28097, Abstract: scheme C keeps routes and texts because its result does not
+ * depend on the order of the expert terms). Same arguments and masking as moe_combine;
+ * per output element the terms w_j * y[dest_row[t,j]] (formed exactly in double) and
+ * y_shared[t] are summed in double in a canonical order -- ascending magnitude, the
+ * negative of two equal magnitudes first -- then rounded to fp32 and to bf16 (nearest
+ * even). Any permutation of a token's (topk_w, dest_row) pairs gives the same bits.
+ * An alternative to the contract's rank-order combine, not used by moe_forward.
+ */
+MOE_API int moe_combine_invariant(const moe_cfg* cfg, const uint16_t* y, const float* topk_w,
+                                  const int32_t* dest_row, const uint16_t* y_shared,
+                                  const uint8_t* token_mask, uint16_t* out, void* stream);
+
+/*
  * The whole layer (SpecForge PR #1003, layer.py: MoELayer = router + routed experts +
  * optional shared expert): moe_route -> moe_permute -> moe_grouped_ffn -> moe_combine
  * on one stream, intermediates in `ws`.
@@ -238,6 +253,24 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
                         float* logits, int32_t* topk_ids, float* topk_w, int32_t* offsets,
                         int32_t* status, void* ws, size_t ws_bytes, void* const* stage_events,
                         void* stream);
+
+/*
+ * Router statistics of one routed batch (SpecForge PR #1003, the load-balance commit: a
+ * Switch-style load-balance value E * sum_e load_e * mean_prob_e over the kept tokens,
+ * K when balanced, with scores L1-normalised per token). Over the N tokens with
+ * token_mask != 0 (all when NULL):
+ *   tokens_per_expert[e] = offsets[e+1] - offsets[e]          (from moe_permute/moe_forward)
+ *   mean_prob[e] = (1/N) sum_t s[t,e] / sum_e' s[t,e']  (s: unbiased scores of `logits`)
+ *   aux = E * sum_e (tokens_per_expert[e] / N) * mean_prob[e]
+ * fp32, summed in a fixed order (deterministic for a given T, no atomics); N == 0 gives 0.
+ *  logits [T,E] fp32, token_mask [T] uint8 or NULL, offsets [E+1] int32 (device);
+ *  tokens_per_expert [E] int32, mean_prob [E] fp32, aux [1] fp32 (device, out);
+ *  ws   moe_workspace_bytes(cfg, MOE_STAGE_STATS) bytes.
+ */
+MOE_API int moe_router_stats(const moe_cfg* cfg, const float* logits, const uint8_t* token_mask,
+                             const int32_t* offsets, int32_t* tokens_per_expert,
+                             float* mean_prob, float* aux, void* ws, size_t ws_bytes,
+                             void* stream);
 
 /*
  * The whole layer from and to HOST memory, overlapping the transfers with the compute

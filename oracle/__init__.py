@@ -72,6 +72,8 @@ _SIGS = {
                                 _P, _I, _P]),
     "oracle_layer_forward": (None, [_I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _I, _P, _P, _P]),
+    "oracle_router_stats": (None, [_I, _I, _I, _P, _P, _P, _I, _P, _P, _P]),
+    "oracle_combine_invariant": (None, [_I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "oracle_num_threads": (_I, []),
 }
 
@@ -204,6 +206,21 @@ def combine_fp32(y, w, dest_row, y_shared=None, mask=None) -> np.ndarray:
     return out
 
 
+def combine_invariant(y, w, dest_row, y_shared=None, mask=None) -> np.ndarray:
+    """Order-invariant combine (canonical-order double sum of exact products); bf16 bits."""
+    y = _arr(y, np.uint16)
+    w = _arr(w, np.float32)
+    d = _arr(dest_row, np.int32)
+    T, K = w.shape
+    H = y.shape[-1]
+    ys = _arr(y_shared, np.uint16)
+    m = _arr(mask, np.uint8)
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_combine_invariant(T, K, H, _ptr(y), _ptr(w), _ptr(d), _ptr(ys), _ptr(m),
+                                   _ptr(out))
+    return out
+
+
 def logits64(x, w_router, logit_bias=None) -> np.ndarray:
     x = _arr(x, np.uint16)
     wr = _arr(w_router, np.uint16)
@@ -283,6 +300,21 @@ def layer_forward(shape, tensors, sel):
                                _ptr(lb), _ptr(sb), _ptr(w13), _ptr(w2), _ptr(w13s), _ptr(w2s),
                                n, _ptr(s), _ptr(ids), _ptr(out))
     return ids, out
+
+
+def router_stats(logits, ids, score_fn: int, mask=None):
+    """(counts [E] int64, mean_prob [E] float64, aux float) of one routed batch."""
+    l = _arr(logits, np.float32)
+    ids = _arr(ids, np.int32)
+    m = _arr(mask, np.uint8)
+    T, E = l.shape
+    K = ids.shape[1]
+    counts = np.empty(E, np.int64)
+    mp = np.empty(E, np.float64)
+    aux = np.zeros(1, np.float64)
+    lib().oracle_router_stats(T, E, K, _ptr(l), _ptr(ids), _ptr(m), score_fn, _ptr(counts),
+                              _ptr(mp), _ptr(aux))
+    return counts, mp, float(aux[0])
 
 
 def num_threads() -> int:

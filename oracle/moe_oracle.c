@@ -468,3 +468,102 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------ router statistics */
+/*
+ * Router statistics of one forward (SpecForge PR #1003, the load-balance commit: a
+ * Switch-style load-balance value E * sum_e load_e * mean_prob_e over the kept tokens,
+ * equal to K when balanced; scores L1-normalised per token so sigmoid and softmax routers
+ * share the formula; padding skipped through the token mask). Reading: over the N kept
+ * tokens, count_e = assignments routed to e, load_e = count_e / N, p_{t,e} = s_{t,e} /
+ * sum_e' s_{t,e'} with s the unbiased scores of the fp32 logits (computed here in
+ * double), mean_prob_e = sum_t p_{t,e} / N, aux = E * sum_e load_e * mean_prob_e.
+ * With N == 0: counts 0, mean_prob 0, aux 0.
+ */
+void oracle_router_stats(int T, int E, int K, const float* logits, const int32_t* ids,
+                         const uint8_t* mask, int score_fn, int64_t* counts, double* mean_prob,
+                         double* aux)
+{
+    int64_t n = 0;
+    for (int e = 0; e < E; ++e) { counts[e] = 0; mean_prob[e] = 0.0; }
+    double* s = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int t = 0; t < T; ++t) {
+        if (mask && !mask[t]) continue;
+        n += 1;
+        for (int j = 0; j < K; ++j) {
+            int32_t e = ids[(int64_t)t * K + j];
+            if (e >= 0 && e < E) counts[e] += 1;
+        }
+        const float* l = logits + (int64_t)t * E;
+        double tot = 0.0;
+        if (score_fn == ORACLE_SIGMOID) {
+            for (int e = 0; e < E; ++e) s[e] = 1.0 / (1.0 + exp(-(double)l[e]));
+        } else {
+            double m = -INFINITY;
+            for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = (double)l[e];
+            for (int e = 0; e < E; ++e) s[e] = exp((double)l[e] - m);
+        }
+        for (int e = 0; e < E; ++e) tot += s[e];
+        for (int e = 0; e < E; ++e) mean_prob[e] += s[e] / tot;
+    }
+    free(s);
+    double a = 0.0;
+    if (n > 0) {
+        for (int e = 0; e < E; ++e) {
+            mean_prob[e] /= (double)n;
+            a += ((double)counts[e] / (double)n) * mean_prob[e];
+        }
+        a *= (double)E;
+    }
+    *aux = a;
+}
+
+/* ------------------------------------------------------------------ order-invariant combine */
+/*
+ * An order-invariant weighted combine ("From Expert Reduction to Behavioral Divergence",
+ * arXiv 2607.28097, Abstract: scheme C keeps routes and texts because its result does not
+ * depend on the order of the expert terms). Reading: the terms are the products
+ * p_j = w_j * float(y_j) formed exactly in double (24 x 8 significant bits) and, when
+ * given, the shared expert's float(y_shared); they are added in double in a canonical
+ * order -- ascending magnitude, a negative term before the positive one of the same
+ * magnitude -- so the sum is a function of the multiset of terms only; out =
+ * bf16_rne(fp32_rne(sum)). Terms with dest_row < 0 are skipped; masked tokens give 0;
+ * no term gives +0.
+ */
+static int canon_less(double a, double b)
+{
+    double fa = fabs(a), fb = fabs(b);
+    if (fa != fb) return fa < fb;
+    return a < b; /* -x before +x */
+}
+
+void oracle_combine_invariant(int T, int K, int H, const uint16_t* y, const float* w,
+                              const int32_t* dest_row, const uint16_t* y_shared,
+                              const uint8_t* mask, uint16_t* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        uint16_t* o = out + (int64_t)t * H;
+        if (mask && !mask[t]) { for (int h = 0; h < H; ++h) o[h] = 0; continue; }
+        double term[33];
+        for (int h = 0; h < H; ++h) {
+            int n = 0;
+            for (int j = 0; j < K; ++j) {
+                int32_t r = dest_row[(int64_t)t * K + j];
+                if (r < 0) continue;
+                term[n++] = (double)w[(int64_t)t * K + j] *
+                            (double)oracle_bf16_to_f32(y[(int64_t)r * H + h]);
+            }
+            if (y_shared) term[n++] = (double)oracle_bf16_to_f32(y_shared[(int64_t)t * H + h]);
+            for (int i = 1; i < n; ++i) { /* insertion sort into the canonical order */
+                double v = term[i];
+                int k = i - 1;
+                while (k >= 0 && canon_less(v, term[k])) { term[k + 1] = term[k]; --k; }
+                term[k + 1] = v;
+            }
+            double s = 0.0;
+            for (int i = 0; i < n; ++i) s += term[i];
+            o[h] = oracle_f32_to_bf16((float)s);
+        }
+    }
+}

@@ -189,3 +189,56 @@ def test_route_injected_near_ties_bit_exact(name, T, n_near):
     n = near_tie_count(l, s, bias)
     print(f"\n{name}: {n} of {T} tokens with K-th/(K+1)-th choices within 1 ulp")
     assert n >= n_near // 2
+
+
+@pytest.mark.parametrize("name,T,keep", [("qwen3_30b_a3b", 4096, None), ("qwen3_30b_a3b", 3001, 0.8),
+                                         ("dsv_sigmoid", 2048, 0.9), ("tiny", 64, None),
+                                         ("dspark", 1000, 0.5)])
+def test_router_stats_against_oracle(name, T, keep):
+    """tokens_per_expert exact, mean_prob and the load-balance value within fp32 summation
+    error of the FP64 oracle; the same call twice gives the same bits."""
+    s = synthetic.shape(name, T=T)
+    l = synthetic.random_logits(T, s.E, seed=T + s.E, std=1.5)
+    mask = None if keep is None else synthetic.random_mask(T, keep, 21)
+    cfg = moe.Config.of(s)
+    _, ids, _ = moe.route(cfg, logits=l.to(DEV), token_mask=None if mask is None else mask.to(DEV))
+    offsets, _, _, _ = moe.permute(cfg, ids)
+    st1 = moe.router_stats(cfg, l.to(DEV), offsets, None if mask is None else mask.to(DEV))
+    st2 = moe.router_stats(cfg, l.to(DEV), offsets, None if mask is None else mask.to(DEV))
+    r_counts, r_mp, r_aux = oracle.router_stats(l.numpy(), ids.cpu().numpy(), s.score_fn,
+                                                mask=None if mask is None else mask.numpy())
+    assert np.array_equal(st1["tokens_per_expert"].cpu().numpy(), r_counts)
+    assert np.allclose(st1["mean_prob"].cpu().numpy(), r_mp, rtol=2e-4, atol=1e-7)
+    assert abs(float(st1["aux"]) - r_aux) <= 2e-4 * abs(r_aux)
+    for k in st1:
+        assert np.array_equal(bits(st1[k]), bits(st2[k]))
+
+
+@pytest.mark.parametrize("T,K,H,shared,masked", [(64, 2, 128, False, True), (1000, 8, 2048, False, True),
+                                                  (333, 6, 4096, True, True), (100, 16, 256, True, False),
+                                                  (500, 1, 512, False, False)])
+def test_combine_invariant_bit_exact_and_order_free(T, K, H, shared, masked):
+    """The order-invariant combine matches the oracle bit for bit, and permuting each
+    token's (weight, row) pairs does not change a bit (the rank-order combine does)."""
+    rng = np.random.default_rng(T * 11 + K)
+    rows = T * K
+    y = (synthetic.normal_bf16(rows, H, 1.0, T + K, "x").float()
+         * torch.from_numpy(10.0 ** rng.uniform(-2, 2, (rows, 1))).float()).to(torch.bfloat16)
+    ys = synthetic.normal_bf16(T, H, 1.0, T + K, "fill") if shared else None
+    w = rng.uniform(0, 1, (T, K)).astype(np.float32)
+    dest = rng.permutation(rows).astype(np.int32).reshape(T, K)
+    mask = (rng.random(T) > 0.2).astype(np.uint8) if masked else None
+    if masked:
+        dest[mask == 0] = -1
+    cfg = moe.Config(T=T, H=H, E=max(K, 8), K=K, I=128)
+    dev = lambda a: None if a is None else (a if torch.is_tensor(a) else torch.from_numpy(a)).to(DEV)
+    out = moe.combine(cfg, dev(y), dev(w), dev(dest), y_shared=dev(ys), token_mask=dev(mask),
+                      order_invariant=True)
+    ref = oracle.combine_invariant(y, w, dest, ys, mask)
+    assert np.array_equal(bits(out), ref)
+    perm = np.argsort(rng.random((T, K)), axis=1)
+    w2 = np.take_along_axis(w, perm, 1)
+    d2 = np.take_along_axis(dest, perm, 1)
+    out2 = moe.combine(cfg, dev(y), dev(w2), dev(d2), y_shared=dev(ys), token_mask=dev(mask),
+                       order_invariant=True)
+    assert np.array_equal(bits(out2), bits(out))

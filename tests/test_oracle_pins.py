@@ -435,3 +435,86 @@ def test_layer_forward_consistent_with_pieces():
     w64 = oracle.weights64(l64, ids2, s.score_fn, s.renorm)
     ref = oracle.forward64(d["x"], ids2, w64, d["w13"], d["w2"], sel=sel)
     assert np.allclose(out, ref, rtol=1e-14, atol=0)
+
+
+# ------------------------------------------------------------------ router statistics
+
+def test_router_stats_balanced_is_K():
+    # every token routed to K distinct experts, expert loads and mean scores uniform
+    E, K, T = 8, 2, 16
+    l = np.zeros((T, E), F32)  # uniform scores: mean_prob = 1/E
+    ids = np.array([[(2 * t) % E, (2 * t + 1) % E] for t in range(T)], np.int32)
+    counts, mp, aux = oracle.router_stats(l, ids, oracle.SOFTMAX)
+    assert counts.tolist() == [4] * E and np.allclose(mp, 1 / E)
+    assert aux == pytest.approx(K, abs=1e-12)
+
+
+def test_router_stats_hand_worked():
+    # E=2, K=1, two kept tokens and one padding token. Token 0: sigmoid scores of logits
+    # (0, 0) -> (1/2, 1/2), routed to 0; token 1: logits (+inf-ish 20, -20) -> p ~ (1, 0),
+    # routed to 0. load = (1, 0); mean_prob_0 = (1/2 + p) / 2 ~ 3/4; aux = 2 * 1 * 3/4 = 1.5
+    l = np.array([[0, 0], [20, -20], [5, 5]], F32)
+    ids = np.array([[0], [0], [1]], np.int32)
+    mask = np.array([1, 1, 0], np.uint8)
+    counts, mp, aux = oracle.router_stats(l, ids, oracle.SIGMOID, mask=mask)
+    p1 = (1 / (1 + np.exp(-20.0))) / (1 / (1 + np.exp(-20.0)) + 1 / (1 + np.exp(20.0)))
+    assert counts.tolist() == [2, 0]
+    assert mp[0] == pytest.approx((0.5 + p1) / 2, rel=1e-14)
+    assert aux == pytest.approx(2 * 1.0 * (0.5 + p1) / 2, rel=1e-14)
+
+
+def test_router_stats_matches_numpy():
+    rng = np.random.default_rng(13)
+    T, E, K = 300, 16, 3
+    l = (rng.standard_normal((T, E)) * 2).astype(F32)
+    ids, _, _ = oracle.route_fp32(l, K, oracle.SOFTMAX, True)
+    mask = (rng.random(T) > 0.2).astype(np.uint8)
+    counts, mp, aux = oracle.router_stats(l, ids, oracle.SOFTMAX, mask=mask)
+    keep = mask == 1
+    p = softmax64(l[keep])
+    ref_counts = np.bincount(ids[keep].reshape(-1), minlength=E)
+    assert np.array_equal(counts, ref_counts)
+    assert np.allclose(mp, p.mean(0), rtol=1e-12)
+    assert aux == pytest.approx(E * np.sum(ref_counts / keep.sum() * p.mean(0)), rel=1e-12)
+    assert counts.sum() == K * keep.sum() and mp.sum() == pytest.approx(1.0)
+
+
+# ------------------------------------------------------------------ order-invariant combine
+
+def test_combine_invariant_all_720_orders_identical():
+    rng = np.random.default_rng(14)
+    K, H = 6, 64
+    for trial in range(3):
+        w = rng.uniform(0.05, 0.4, (1, K)).astype(F32)
+        y = oracle.f32_to_bf16((rng.standard_normal((K, H)) * 10 ** rng.uniform(-3, 3, (K, 1)))
+                               .astype(F32))
+        d = np.arange(K, dtype=np.int32)[None]
+        ref = oracle.combine_invariant(y, w, d)
+        for perm in itertools.permutations(range(K)):
+            p = list(perm)
+            assert np.array_equal(oracle.combine_invariant(y[p], w[:, p], d), ref)
+        # while the rank-order contract combine does depend on the order here
+        outs = {oracle.combine_acc_fp32(y[list(pp)], w[:, list(pp)], d).tobytes()
+                for pp in itertools.permutations(range(K))}
+        assert len(outs) > 1
+
+
+def test_combine_invariant_cancellation_and_accuracy(golden):
+    c = golden("tree_sum_and_combine_order.json")["combine_case"]
+    w = np.array(c["w"], F32)
+    y = oracle.f32_to_bf16(np.array(c["y"], F32))
+    d = np.array(c["dest_row"], np.int32)
+    # terms 2^24, 1, -2^24: the canonical order adds 1 first, then -2^24 + 2^24 exactly
+    out = oracle.bf16_to_f32(oracle.combine_invariant(y, w, d))
+    assert out.tolist() == [[1.0]]
+    # random rows: within one bf16 rounding (plus fp32) of the float64 sum
+    rng = np.random.default_rng(15)
+    T, K, H = 30, 8, 64
+    w = rng.uniform(0, 0.3, (T, K)).astype(F32)
+    y = oracle.f32_to_bf16(rng.standard_normal((T * K, H)).astype(F32))
+    ys = oracle.f32_to_bf16(rng.standard_normal((T, H)).astype(F32))
+    d = rng.permutation(T * K).astype(np.int32).reshape(T, K)
+    got = oracle.bf16_to_f32(oracle.combine_invariant(y, w, d, ys)).astype(np.float64)
+    yf = oracle.bf16_to_f32(y).astype(np.float64)
+    ref = np.einsum("tk,tkh->th", w.astype(np.float64), yf[d]) + oracle.bf16_to_f32(ys)
+    assert np.all(np.abs(got - ref) <= 2.0**-8 * np.abs(ref) + 1e-30)
