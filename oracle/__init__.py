@@ -62,6 +62,8 @@ _SIGS = {
     "oracle_scores_fp32": (None, [_I, _P, _I, _P]),
     "oracle_select_key": (ctypes.c_uint64, [_F, _I]),
     "oracle_route_fp32": (None, [_I, _I, _I, _P, _P, _P, _I, _I, _F, _P, _P, _P]),
+    "oracle_route_fp32_grouped": (None, [_I, _I, _I, _P, _P, _P, _I, _I, _F, _I, _I, _P, _P,
+                                         _P]),
     "oracle_permute": (_I64, [_I, _I, _I, _P, _P, _P, _P]),
     "oracle_combine_acc_fp32": (None, [_I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "oracle_combine_fp32": (None, [_I, _I, _I, _P, _P, _P, _P, _P, _P]),
@@ -151,8 +153,9 @@ def select_key(c: float, idx: int) -> int:
 
 
 def route_fp32(logits, K: int, score_fn: int, renorm: bool, route_scale: float = 1.0,
-               sel_bias=None, mask=None):
-    """FP32-contract routing. Returns (ids [T,K] int32, w [T,K] fp32, status [2] int64)."""
+               sel_bias=None, mask=None, n_group: int = 0, topk_group: int = 0):
+    """FP32-contract routing (group-limited when n_group > 1). Returns (ids [T,K] int32,
+    w [T,K] fp32, status [2] int64)."""
     l = _arr(logits, np.float32)
     T, E = l.shape
     sb = _arr(sel_bias, np.float32)
@@ -160,8 +163,9 @@ def route_fp32(logits, K: int, score_fn: int, renorm: bool, route_scale: float =
     ids = np.empty((T, K), np.int32)
     w = np.empty((T, K), np.float32)
     st = np.zeros(2, np.int64)
-    lib().oracle_route_fp32(T, E, K, _ptr(l), _ptr(sb), _ptr(m), score_fn, int(bool(renorm)),
-                            float(route_scale), _ptr(ids), _ptr(w), _ptr(st))
+    lib().oracle_route_fp32_grouped(T, E, K, _ptr(l), _ptr(sb), _ptr(m), score_fn,
+                                    int(bool(renorm)), float(route_scale), int(n_group),
+                                    int(topk_group), _ptr(ids), _ptr(w), _ptr(st))
     return ids, w, st
 
 

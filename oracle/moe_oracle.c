@@ -185,9 +185,46 @@ uint64_t oracle_select_key(float c, int id)
  * Masked tokens (mask[t] == 0) get ids -1 and weights 0.
  * status[0] += tokens with a NaN choice, status[1] += zero-denominator tokens.
  */
-void oracle_route_fp32(int T, int E, int K, const float* logits, const float* sel_bias,
-                       const uint8_t* mask, int score_fn, int renorm, float route_scale,
-                       int32_t* ids, float* w, int64_t* status)
+/*
+ * Group-limited selection (the DeepSeek family's override of `select` named in SpecForge
+ * PR #1003, "Out of scope" and the select() refactor note; the pages give no formula).
+ * Reading: the E experts form n_group contiguous groups of E / n_group; a group's score is
+ * the fp32 sum of its two best choices (best + second, by the selection key; one choice
+ * when the group has one expert); the topk_group groups with the largest (group score,
+ * then lower group id) are kept; the K experts are then chosen among the kept groups only.
+ * n_group <= 1 turns it off. Weights still come from the unbiased scores.
+ */
+static void keep_groups(int E, int n_group, int topk_group, const float* c,
+                        const uint64_t* key, unsigned char* excluded)
+{
+    const int gs = E / n_group;
+    uint64_t* gkey = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)n_group);
+    unsigned char* kept = (unsigned char*)calloc((size_t)n_group, 1);
+    for (int g = 0; g < n_group; ++g) {
+        int b1 = -1, b2 = -1;
+        for (int e = g * gs; e < (g + 1) * gs; ++e) {
+            if (b1 < 0 || key[e] > key[b1]) { b2 = b1; b1 = e; }
+            else if (b2 < 0 || key[e] > key[b2]) { b2 = e; }
+        }
+        float score = c[b1];
+        if (b2 >= 0) score = score + c[b2];
+        gkey[g] = oracle_select_key(score, g);
+    }
+    for (int r = 0; r < topk_group; ++r) {
+        int best = -1;
+        for (int g = 0; g < n_group; ++g)
+            if (!kept[g] && (best < 0 || gkey[g] > gkey[best])) best = g;
+        kept[best] = 1;
+    }
+    for (int e = 0; e < E; ++e) excluded[e] = !kept[e / gs];
+    free(gkey);
+    free(kept);
+}
+
+void oracle_route_fp32_grouped(int T, int E, int K, const float* logits, const float* sel_bias,
+                               const uint8_t* mask, int score_fn, int renorm, float route_scale,
+                               int n_group, int topk_group, int32_t* ids, float* w,
+                               int64_t* status)
 {
     int64_t nan_tokens = 0, zero_den = 0;
 #pragma omp parallel for reduction(+ : nan_tokens, zero_den) schedule(static)
@@ -199,6 +236,7 @@ void oracle_route_fp32(int T, int E, int K, const float* logits, const float* se
             continue;
         }
         float* s = (float*)malloc(sizeof(float) * (size_t)E);
+        float* cv = (float*)malloc(sizeof(float) * (size_t)E);
         uint64_t* key = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)E);
         unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
         oracle_scores_fp32(E, logits + (int64_t)t * E, score_fn, s);
@@ -206,9 +244,11 @@ void oracle_route_fp32(int T, int E, int K, const float* logits, const float* se
         for (int e = 0; e < E; ++e) {
             float c = sel_bias ? s[e] + sel_bias[e] : s[e];
             if (isnan(c)) has_nan = 1;
+            cv[e] = c;
             key[e] = oracle_select_key(c, e);
         }
         nan_tokens += has_nan;
+        if (n_group > 1) keep_groups(E, n_group, topk_group, cv, key, taken);
         for (int j = 0; j < K; ++j) {
             int best = -1;
             for (int e = 0; e < E; ++e)
@@ -228,9 +268,17 @@ void oracle_route_fp32(int T, int E, int K, const float* logits, const float* se
         } else {
             for (int j = 0; j < K; ++j) wt[j] = s[id[j]] * route_scale;
         }
-        free(s); free(key); free(taken);
+        free(s); free(cv); free(key); free(taken);
     }
     if (status) { status[0] += nan_tokens; status[1] += zero_den; }
+}
+
+void oracle_route_fp32(int T, int E, int K, const float* logits, const float* sel_bias,
+                       const uint8_t* mask, int score_fn, int renorm, float route_scale,
+                       int32_t* ids, float* w, int64_t* status)
+{
+    oracle_route_fp32_grouped(T, E, K, logits, sel_bias, mask, score_fn, renorm, route_scale, 0,
+                              0, ids, w, status);
 }
 
 /* ------------------------------------------------------------------ permutation */

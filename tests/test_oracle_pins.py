@@ -518,3 +518,55 @@ def test_combine_invariant_cancellation_and_accuracy(golden):
     yf = oracle.bf16_to_f32(y).astype(np.float64)
     ref = np.einsum("tk,tkh->th", w.astype(np.float64), yf[d]) + oracle.bf16_to_f32(ys)
     assert np.all(np.abs(got - ref) <= 2.0**-8 * np.abs(ref) + 1e-30)
+
+
+# ------------------------------------------------------------------ group-limited selection
+
+def brute_force_grouped(choice, K, n_group, topk_group):
+    """Group scores = best + second-best choice of each group (by the selection key), the
+    topk_group best groups kept (higher score, then lower group), then the brute-force
+    top-K over the kept experts (excluded experts never chosen)."""
+    E = len(choice)
+    gs = E // n_group
+    gkeys = []
+    for g in range(n_group):
+        members = sorted(range(g * gs, (g + 1) * gs), key=lambda e: py_key(choice[e], e),
+                         reverse=True)
+        sc = np.float32(choice[members[0]])
+        if gs > 1:
+            sc = np.float32(sc + np.float32(choice[members[1]]))
+        gkeys.append((py_key(sc, g), g))
+    kept = {g for _, g in sorted(gkeys, reverse=True)[:topk_group]}
+    masked = [choice[e] if e // gs in kept else None for e in range(E)]
+    best, best_key = None, None
+    for tup in itertools.permutations([e for e in range(E) if masked[e] is not None], K):
+        key = tuple(py_key(choice[e], e) for e in tup)
+        if best_key is None or key > best_key:
+            best, best_key = tup, key
+    return list(best)
+
+
+@pytest.mark.parametrize("E,K,n_group,topk_group", [(8, 2, 4, 2), (9, 3, 3, 1), (10, 3, 5, 3),
+                                                    (8, 2, 8, 3), (6, 2, 2, 2)])
+def test_grouped_route_brute_force(E, K, n_group, topk_group):
+    rng = np.random.default_rng(E * 100 + K * 10 + n_group)
+    for trial in range(25):
+        l = (rng.standard_normal(E) * 2).astype(F32)
+        if trial % 5 == 1:
+            l[:] = F32(0.3)                      # all tied: lowest groups, lowest ids
+        if trial % 5 == 2:
+            i, j = rng.choice(E, 2, replace=False)
+            l[j] = l[i]
+        bias = rng.uniform(-0.05, 0.05, E).astype(F32) if trial % 2 else None
+        score_fn = oracle.SIGMOID if trial % 3 == 0 else oracle.SOFTMAX
+        ids, w, _ = oracle.route_fp32(l[None], K, score_fn, True, 1.0, sel_bias=bias,
+                                      n_group=n_group, topk_group=topk_group)
+        s = oracle.scores_fp32(l, score_fn)
+        choice = s if bias is None else (s + bias).astype(F32)
+        assert list(ids[0]) == brute_force_grouped(list(choice), K, n_group, topk_group)
+    # n_group = 1 or topk_group = n_group leaves plain top-K
+    l = (rng.standard_normal((20, E)) * 2).astype(F32)
+    a = oracle.route_fp32(l, K, oracle.SOFTMAX, True)[0]
+    assert np.array_equal(oracle.route_fp32(l, K, oracle.SOFTMAX, True, n_group=1)[0], a)
+    assert np.array_equal(oracle.route_fp32(l, K, oracle.SOFTMAX, True, n_group=n_group,
+                                            topk_group=n_group)[0], a)
