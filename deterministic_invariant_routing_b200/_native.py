@@ -43,7 +43,8 @@ class MoeCfg(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("K", ctypes.c_int32), ("I", ctypes.c_int32), ("I_shared", ctypes.c_int32),
                 ("score_fn", ctypes.c_int32), ("renorm", ctypes.c_int32),
-                ("route_scale", ctypes.c_float)]
+                ("route_scale", ctypes.c_float), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p

@@ -52,6 +52,12 @@ int check_cfg(const moe_cfg* c)
     if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_SHAPE;
     if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_SHAPE;
     if (!isfinite(c->route_scale)) return MOE_ERR_SHAPE;
+    if (c->n_group < 0 || c->n_group > 32) return MOE_ERR_SHAPE;
+    if (c->n_group > 1) {
+        if (c->E % c->n_group != 0 || c->topk_group < 1 || c->topk_group > c->n_group ||
+            c->K > c->topk_group * (c->E / c->n_group))
+            return MOE_ERR_SHAPE;
+    }
     return MOE_OK;
 }
 
@@ -336,7 +342,7 @@ using namespace moe;
 
 extern "C" {
 
-MOE_API int moe_abi_version(void) { return 100; }
+MOE_API int moe_abi_version(void) { return 101; }
 
 MOE_API const char* moe_status_string(int code)
 {

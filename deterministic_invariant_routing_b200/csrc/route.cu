@@ -10,6 +10,12 @@
 // the softmax denominator is the 32-lane tree (lane L sums experts L, L+32, ... in
 // increasing order, then butterfly levels 16, 8, 4, 2, 1); the selection compares
 // 64-bit keys (ordered choice bits, then inverted id), so ties go to the lower id.
+//
+// Group-limited selection (n_group > 1, the DeepSeek family's override of the selection
+// named in SpecForge PR #1003): the warp stages the token's choice values in shared
+// memory, lane g scans group g in expert order for its two best keys and scores the group
+// by their fp32 sum, topk_group warp arg-max rounds over the group keys pick the kept
+// groups, and the experts of the other groups get key 0 before the K selection rounds.
 #include "route_math.cuh"
 
 namespace moe {
@@ -20,16 +26,35 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
     return a > b ? a : b;
 }
 
+__device__ __forceinline__ unsigned long long select_key(float c, int id)
+{
+    return ((unsigned long long)order_bits(c) << 32) |
+           (unsigned long long)(0xffffffffu - (uint32_t)id);
+}
+
+// warp arg-max of 64-bit keys as two 32-bit reductions: the highest choice bits, then,
+// among the lanes holding them, the highest inverted id; returns the id
+__device__ __forceinline__ int warp_argmax_id(unsigned long long k)
+{
+    const uint32_t hi = (uint32_t)(k >> 32), lo = (uint32_t)k;
+    const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+    return (int)(0xffffffffu - mlo);
+}
+
 // NE = experts held per lane (E <= 32 * NE)
 template <int NE>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
                                                     int K, const float* __restrict__ sel_bias,
                                                     const uint8_t* __restrict__ mask, int score_fn,
                                                     int renorm, float route_scale,
+                                                    int n_group, int topk_group,
                                                     int32_t* __restrict__ ids,
                                                     float* __restrict__ w, int32_t* status)
 {
+    extern __shared__ float choice_smem[];  // [warps][E], group-limited selection only
     const int lane = threadIdx.x & 31;
+    float* cw = choice_smem + (threadIdx.x >> 5) * E;
     const int warps_per_block = blockDim.x >> 5;
     int nan_tokens = 0, zero_den = 0;
     for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
@@ -85,13 +110,41 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             if (e < E) {
                 const float c = (sel_bias != nullptr) ? __fadd_rn(s[i], sel_bias[e]) : s[i];
                 any_nan |= isnan(c);
-                key[i] = ((unsigned long long)order_bits(c) << 32) |
-                         (unsigned long long)(0xffffffffu - (uint32_t)e);
+                key[i] = select_key(c, e);
+                if (n_group > 1) cw[e] = c;
             } else {
                 key[i] = 0ull;
             }
         }
         if (__any_sync(0xffffffffu, any_nan)) nan_tokens += (lane == 0);
+        if (n_group > 1) {
+            __syncwarp();
+            const int gs = E / n_group;
+            unsigned long long gk = 0ull;
+            if (lane < n_group) {
+                unsigned long long k1 = 0ull, k2 = 0ull;
+                float c1 = 0.0f, c2 = 0.0f;
+                for (int e = lane * gs; e < (lane + 1) * gs; ++e) {
+                    const float c = cw[e];
+                    const unsigned long long k = select_key(c, e);
+                    if (k > k1) { k2 = k1; c2 = c1; k1 = k; c1 = c; }
+                    else if (k > k2) { k2 = k; c2 = c; }
+                }
+                gk = select_key(gs > 1 ? __fadd_rn(c1, c2) : c1, lane);
+            }
+            __syncwarp();  // the scan is done before the next token overwrites cw
+            uint32_t kept = 0u;
+            for (int r = 0; r < topk_group; ++r) {
+                const int g = warp_argmax_id(gk);
+                kept |= 1u << g;
+                if (lane == g) gk = 0ull;
+            }
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E && ((kept >> (e / gs)) & 1u) == 0u) key[i] = 0ull;
+            }
+        }
         // K rounds of a warp-wide arg-max over the remaining keys
         int my_id = -1;
         float my_s = 0.0f, den = 0.0f;
@@ -99,12 +152,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             unsigned long long best = 0ull;
 #pragma unroll
             for (int i = 0; i < NE; ++i) best = umax64(best, key[i]);
-            // warp arg-max of the 64-bit keys as two 32-bit reductions: the highest choice
-            // bits, then, among the lanes holding them, the highest inverted id
-            const uint32_t hi = (uint32_t)(best >> 32), lo = (uint32_t)best;
-            const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-            const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
-            const int e = (int)(0xffffffffu - mlo);
+            const int e = warp_argmax_id(best);
             const int owner = e & 31, slot = e >> 5;
             float se = 0.0f;
 #pragma unroll
@@ -144,9 +192,11 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bi
     int blocks = (c.T + wpb - 1) / wpb;
     const int cap = num_sms() * 8;
     if (blocks > cap) blocks = cap;
-    route_kernel<NE><<<blocks, threads, 0, st>>>(logits, c.T, c.E, c.K, sel_bias, mask,
-                                                 c.score_fn, c.renorm, c.route_scale, ids, w,
-                                                 status);
+    const int n_group = c.n_group > 1 ? c.n_group : 0;
+    const size_t smem = n_group ? (size_t)wpb * c.E * sizeof(float) : 0;
+    route_kernel<NE><<<blocks, threads, smem, st>>>(logits, c.T, c.E, c.K, sel_bias, mask,
+                                                    c.score_fn, c.renorm, c.route_scale, n_group,
+                                                    c.topk_group, ids, w, status);
     return cudaGetLastError();
 }
 

@@ -46,20 +46,25 @@ class Config:
     score_fn: int = SOFTMAX
     renorm: bool = True
     route_scale: float = 1.0
+    n_group: int = 0        # group-limited selection, 0 = off
+    topk_group: int = 0
 
     @classmethod
     def of(cls, shape, T: Optional[int] = None) -> "Config":
         """From a workload shape (anything with the same field names)."""
         return cls(T=shape.T if T is None else T, H=shape.H, E=shape.E, K=shape.K, I=shape.I,
                    I_shared=shape.I_shared, score_fn=shape.score_fn, renorm=bool(shape.renorm),
-                   route_scale=float(shape.route_scale))
+                   route_scale=float(shape.route_scale),
+                   n_group=int(getattr(shape, "n_group", 0)),
+                   topk_group=int(getattr(shape, "topk_group", 0)))
 
     def with_T(self, T: int) -> "Config":
         return dataclasses.replace(self, T=T)
 
     def c(self) -> N.MoeCfg:
         return N.MoeCfg(self.T, self.H, self.E, self.K, self.I, self.I_shared, self.score_fn,
-                        int(bool(self.renorm)), float(self.route_scale))
+                        int(bool(self.renorm)), float(self.route_scale), int(self.n_group),
+                        int(self.topk_group))
 
 
 def _p(t: Optional[torch.Tensor]):

@@ -49,6 +49,8 @@ class LayerShape:
     sel_bias_range: Optional[float]   # selection bias ~ U(-r, r), or None
     logit_bias_std: Optional[float]   # per-expert logit skew ~ N(0, s), or None
     seed: int
+    n_group: int = 0                  # group-limited selection (0 = off)
+    topk_group: int = 0
 
 
 WORKLOADS = {

@@ -35,7 +35,7 @@
  *
  * Shapes supported: 1 <= E <= 1024, 1 <= K <= min(E, 16), H % 128 == 0 and
  * 128 <= H <= 16384, I % 128 == 0, I_shared % 128 == 0 (0 = no shared expert),
- * 0 <= T and T * K < 2^31. T == 0 is a no-op.
+ * 0 <= T and T * K < 2^31. T == 0 is a no-op. Group-limited selection: see moe_cfg.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -94,6 +94,19 @@ typedef struct moe_cfg {
     int32_t score_fn;    /* MOE_SOFTMAX or MOE_SIGMOID */
     int32_t renorm;      /* 1: weights renormalised over the K selected scores */
     float route_scale;   /* weights are multiplied by it (1.0 = unchanged) */
+    /*
+     * Group-limited selection (the DeepSeek family's override of the selection step,
+     * SpecForge PR #1003, "Out of scope"; the pages name it without a formula). 0 or 1 =
+     * off. Otherwise the E experts form n_group contiguous groups of E / n_group; a
+     * group's score is the fp32 sum of its two best choices (s + sel_bias, best first,
+     * the tie rule of the selection; one choice when a group has one expert); the
+     * topk_group best groups are kept (higher score, then lower group id) and the K
+     * experts are chosen among the kept groups only. Weights still come from the unbiased
+     * scores. Needs E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group and
+     * K <= topk_group * (E / n_group); anything else is MOE_ERR_SHAPE.
+     */
+    int32_t n_group;
+    int32_t topk_group;
 } moe_cfg;
 
 /*

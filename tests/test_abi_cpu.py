@@ -42,7 +42,7 @@ def test_status_strings(lib):
     assert N.status_string(0) == "ok"
     for code in (-1, -2, -3, -4, -5, -6):
         assert N.status_string(code) != "unknown status"
-    assert lib.moe_abi_version() == 100
+    assert lib.moe_abi_version() == 101
 
 
 GOOD = dict(T=64, H=128, E=8, K=2, I=256)
@@ -57,7 +57,12 @@ def cfg(**over):
 @pytest.mark.parametrize("over", [dict(H=100), dict(H=64), dict(I=100), dict(E=0),
                                   dict(E=1025), dict(K=0), dict(K=17), dict(K=9, E=8),
                                   dict(I_shared=100), dict(T=-1), dict(score_fn=2),
-                                  dict(T=200_000_000, K=16)])
+                                  dict(T=200_000_000, K=16),
+                                  # group-limited selection
+                                  dict(n_group=3, topk_group=1), dict(n_group=4, topk_group=0),
+                                  dict(n_group=4, topk_group=5), dict(n_group=-1),
+                                  dict(n_group=4, topk_group=1, K=3),
+                                  dict(E=64, n_group=64, topk_group=2)])
 def test_bad_shapes_rejected(lib, over):
     c = cfg(**over)
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first

@@ -37,8 +37,8 @@ def sample_tokens(T, n, seed):
     return np.unique(np.clip(np.concatenate([edge, pick]), 0, T - 1)).astype(np.int32)
 
 
-def check_layer(name, T, n_sample=16, keep=None, report=None):
-    s, d, cfg = layer(name, T)
+def check_layer(name, T, n_sample=16, keep=None, report=None, **over):
+    s, d, cfg = layer(name, T, **over)
     mask = None
     if keep is not None:
         mask = synthetic.random_mask(T, keep, 77).to(DEV)
@@ -59,7 +59,8 @@ def check_layer(name, T, n_sample=16, keep=None, report=None):
     # level 1: routes from the GPU's logits, bit-exact
     sb = None if d["sel_bias"] is None else d["sel_bias"].cpu().numpy()
     r_ids, r_w, r_st = oracle.route_fp32(g_logits, s.K, s.score_fn, s.renorm, s.route_scale,
-                                         sel_bias=sb, mask=mask_np)
+                                         sel_bias=sb, mask=mask_np, n_group=s.n_group,
+                                         topk_group=s.topk_group)
     g_ids = r["ids"].cpu().numpy()
     assert np.array_equal(g_ids, r_ids)
     assert np.array_equal(r["w"].cpu().numpy().view(np.uint32), r_w.view(np.uint32))
@@ -150,6 +151,13 @@ def test_dspark_shape():
 
 def test_dsv_sigmoid_shape():
     check_layer("dsv_sigmoid", 8192, n_sample=12)
+
+
+def test_dsv_sigmoid_group_limited():
+    """The DeepSeek-style layer with group-limited selection (8 groups of 32, 4 kept)."""
+    r = check_layer("dsv_sigmoid", 4096, n_sample=12, n_group=8, topk_group=4)
+    ids = r["ids"].cpu().numpy()
+    assert np.all(np.array([len(set(row // 32)) for row in ids]) <= 4)
 
 
 def test_tied_router_rows_pick_lower_id():

@@ -45,6 +45,51 @@ ROUTE_CASES = [
 ]
 
 
+GROUPED_CASES = [
+    # E, K, score_fn, with_bias, n_group, topk_group, T
+    (256, 8, SG, True, 8, 4, 4096),     # DeepSeek-V3-like
+    (64, 6, SM, False, 8, 3, 2000),
+    (1024, 16, SM, True, 32, 4, 517),
+    (96, 4, SG, False, 3, 1, 999),
+    (32, 2, SM, True, 32, 2, 300),      # one expert per group
+    (160, 6, SG, True, 20, 20, 700),    # every group kept: plain top-K
+]
+
+
+@pytest.mark.parametrize("E,K,score_fn,with_bias,n_group,topk_group,T", GROUPED_CASES)
+def test_route_group_limited_bit_exact(E, K, score_fn, with_bias, n_group, topk_group, T):
+    seed = 300 + E + n_group
+    l = adversarial_logits(T, E, seed)
+    gs = E // n_group
+    rng = np.random.default_rng(seed)
+    for t in range(50, min(T, 90)):       # two groups with exactly tied scores
+        g0, g1 = rng.choice(n_group, 2, replace=False)
+        l[t, g1 * gs:(g1 + 1) * gs] = l[t, g0 * gs:(g0 + 1) * gs]
+    bias = synthetic.uniform_f32(E, 0.05, seed, "sel_bias").numpy() if with_bias else None
+    if bias is not None:                  # keep the copied groups' choices tied
+        bias = np.tile(bias[:gs], n_group).astype(np.float32)
+    mask = synthetic.random_mask(T, 0.9, seed).numpy()
+    cfg = moe.Config(T=T, H=128, E=E, K=K, I=128, score_fn=score_fn, renorm=True,
+                     n_group=n_group, topk_group=topk_group)
+    st = moe.new_status(DEV)
+    _, ids, w = moe.route(cfg, logits=torch.from_numpy(l).to(DEV),
+                          sel_bias=None if bias is None else torch.from_numpy(bias).to(DEV),
+                          token_mask=torch.from_numpy(mask).to(DEV), status=st, check=False)
+    torch.cuda.synchronize()
+    r_ids, r_w, r_st = oracle.route_fp32(l, K, score_fn, True, 1.0, sel_bias=bias, mask=mask,
+                                         n_group=n_group, topk_group=topk_group)
+    g_ids = ids.cpu().numpy()
+    assert np.array_equal(g_ids, r_ids), np.argwhere(g_ids != r_ids)[:5]
+    g_w = w.cpu().numpy()
+    nan = np.isnan(r_w)
+    assert np.array_equal(np.isnan(g_w), nan)
+    assert np.array_equal(g_w[~nan].view(np.uint32), r_w[~nan].view(np.uint32))
+    s = st.cpu().numpy()
+    assert s[N.MOE_ST_NAN_TOKENS] == r_st[0] and s[N.MOE_ST_ZERO_DENOM] == r_st[1]
+    live = g_ids[:, 0] >= 0
+    assert all(len(set(row // gs)) <= topk_group for row in g_ids[live])
+
+
 @pytest.mark.parametrize("E,K,score_fn,renorm,scale,with_bias,T", ROUTE_CASES)
 def test_route_bit_exact(E, K, score_fn, renorm, scale, with_bias, T):
     seed = 100 + E + K
