@@ -27,6 +27,11 @@
 // Accumulators: the commit of the last k-block arrives on tfull[a] of both CTAs; each
 // CTA's epilogue drains its own TMEM rows and arrives on the leader's tempty[a] (256
 // arrivals). Every wait is bounded and a give-up is recorded in MOE_ST_PIPE_TIMEOUT.
+//
+// Output: each epilogue warp owns 32 accumulator rows and writes them 32 columns at a time.
+// A block whose 32 rows all lie inside the group goes through a 2 KiB shared-memory tile
+// (64-byte swizzle, two per warp, alternating) and one TMA store; the partial block at a
+// group's end is stored row by row from registers, so no padding row reaches global memory.
 #include <cuda_bf16.h>
 
 #include "tc_common.cuh"
@@ -65,9 +70,10 @@ struct Cfg2 {
     static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
     static constexpr uint32_t kTmemCols = 2 * NP;
     static constexpr int kBars = 2 * kStages + 5;
+    static constexpr uint32_t kEpiBytes = 4 * 2 * 2048;  // 4 warps x 2 tiles of 32 x 32 bf16
     static size_t smem_bytes(int groups)
     {
-        return 1024 + (size_t)kStages * kStageBytes + kBars * 8 + 16 +
+        return 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kBars * 8 + 16 +
                (size_t)2 * (groups + 1) * sizeof(int32_t) + HM * sizeof(int32_t);
     }
 };
@@ -98,7 +104,8 @@ __device__ __forceinline__ PairTile decode_pair_tile(int t, int n_tiles, int gro
 template <int EPI, int NP, bool GATHER>
 __global__ void __launch_bounds__(kThreads2, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, PairArgs args)
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO, PairArgs args)
 {
     using C = Cfg2<EPI, NP>;
     constexpr int S = C::kStages;
@@ -110,7 +117,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
     uint8_t* base = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     const uint32_t sA0 = smem_u32(base);
     const uint32_t sB0 = sA0 + S * kA2Bytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * C::kStageBytes);
+    const uint32_t sE0 = sA0 + S * C::kStageBytes;  // epilogue store tiles
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * C::kStageBytes + C::kEpiBytes);
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(S + s); };
@@ -351,6 +359,39 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const int row = q * 32 + lane;
         const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
         const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
+        const uint32_t ebuf = sE0 + (uint32_t)q * 4096u;
+        uint32_t eb = 0;  // which of the warp's two store tiles is next
+        // this lane's row of a store tile: 64 bytes, 16-byte chunks at the swizzled place
+        const uint32_t erow = (uint32_t)lane * 64u, eswz = ((uint32_t)lane >> 1) & 3u;
+        // 32 x 32 block of rows [row_blk, +32), columns [col, +32): through shared memory
+        // and TMA when the whole block is inside the group, else the valid rows directly
+        auto store_block = [&](const uint32_t (&pk)[16], bool full_blk, bool valid,
+                               int row_blk, int col, uint16_t* dst_row) {
+            if (full_blk) {
+                const uint32_t b = ebuf + eb * 2048u;
+                if (lane == 0) bulk_wait_read<1>();  // the tile stored two blocks ago is read
+                __syncwarp();
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     b + erow + ((((uint32_t)v) ^ eswz) << 4)),
+                                 "r"(pk[4 * v]), "r"(pk[4 * v + 1]), "r"(pk[4 * v + 2]),
+                                 "r"(pk[4 * v + 3])
+                                 : "memory");
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmO, b, col, row_blk);
+                    bulk_commit();
+                }
+                eb ^= 1u;
+            } else if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+        };
         int i = 0;
         for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
             const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
@@ -364,6 +405,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * NP);
             const int64_t grow = ti.row0 + (int64_t)rank * HM + row;
             const bool valid = grow < ti.row_end;
+            const int row_blk = (int)(ti.row0 + (int64_t)rank * HM + q * 32);
+            const bool full_blk = (int64_t)row_blk + 31 < ti.row_end;
             uint16_t* out = static_cast<uint16_t*>(args.out);
             if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
@@ -383,14 +426,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
                         }
                         pk[j] = bf16x2_rne(hv[0], hv[1]);
                     }
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            out + grow * args.ldo + (int64_t)ti.n * (NP / 2) + c);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
-                                                pk[4 * v + 3]);
-                    }
+                    const int col = ti.n * (NP / 2) + c;
+                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
                 }
             } else {
 #pragma unroll 1
@@ -401,19 +438,14 @@ __global__ void __launch_bounds__(kThreads2, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         pk[j] = bf16x2_rne(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo +
-                                                              (int64_t)ti.n * NP + c);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
-                                                pk[4 * v + 3]);
-                    }
+                    const int col = ti.n * NP + c;
+                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
                 }
             }
             tc_fence_before();
             mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
         }
+        if (lane == 0) bulk_wait_all();  // the TMA stores have written global memory
     }
 
     tc_fence_before();
@@ -465,10 +497,12 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
         max_clusters[dev] = n;
         max_smem[dev] = smem;
     }
-    CUtensorMap ma, mb;
+    const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
+    CUtensorMap ma, mb, mo;
     if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) return cudaErrorInvalidValue;
     if (!make_map(&mb, p.b, (int64_t)groups * p.b_rows_per_group, p.k, NP / 2))
         return cudaErrorInvalidValue;
+    if (!make_store_map(&mo, p.out, rows_total, p.n, p.ldo)) return cudaErrorInvalidValue;
     PairArgs a;
     a.k_blocks = p.k / BK;
     a.n_tiles = (EPI == EPI_SWIGLU) ? p.n / (NP / 2) : p.n / NP;
@@ -483,13 +517,12 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.out = p.out;
     a.ldo = p.ldo;
     a.status = p.status;
-    const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
     const int64_t max_tiles = ((rows_total + PM - 1) / PM + groups) * a.n_tiles;
     int64_t clusters = max_clusters[dev];
     if (max_tiles < clusters) clusters = max_tiles;
     if (clusters < 1) clusters = 1;
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, a);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mo, a);
 }
 
 }  // namespace
