@@ -29,6 +29,7 @@ _lib = None
 
 SOFTMAX = 0
 SIGMOID = 1
+SQRTSOFTPLUS = 2
 
 GCC_FLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC",
              "-std=c11", "-Wall"]
@@ -58,6 +59,8 @@ _SIGS = {
     "oracle_f32_to_bf16_array": (None, [_P, _P, _I64]),
     "oracle_exp_rl": (_F, [_F]),
     "oracle_exp_rl_array": (None, [_P, _P, _I64]),
+    "oracle_fn_array": (None, [_I, _P, _P, _I64]),
+    "oracle_sqrtsoftplus64": (_D, [_D]),
     "oracle_tree_sum32": (_F, [_P, _I]),
     "oracle_scores_fp32": (None, [_I, _P, _I, _P]),
     "oracle_select_key": (ctypes.c_uint64, [_F, _I]),
@@ -134,6 +137,34 @@ def exp_rl(x) -> np.ndarray:
     out = np.empty_like(x)
     lib().oracle_exp_rl_array(_ptr(x), _ptr(out), x.size)
     return out
+
+
+def _fn(which, x):
+    x = _arr(x, np.float32)
+    out = np.empty_like(x)
+    lib().oracle_fn_array(which, _ptr(x), _ptr(out), x.size)
+    return out
+
+
+def ln_rl(v) -> np.ndarray:
+    """The contract's fp32 natural log for v >= 1 (the sqrtsoftplus score's log1p)."""
+    return _fn(0, v)
+
+
+def log1p_rl(u) -> np.ndarray:
+    """The contract's fp32 log1p for u >= 0 (Goldberg's formula over ln_rl)."""
+    return _fn(1, u)
+
+
+def sqrtsoftplus_rl(x) -> np.ndarray:
+    """The contract's fp32 sqrtsoftplus score."""
+    return _fn(2, x)
+
+
+def sqrtsoftplus64(x) -> np.ndarray:
+    """sqrt(softplus(x)) in double with libm."""
+    f = lib().oracle_sqrtsoftplus64
+    return np.array([f(float(v)) for v in np.ravel(x)], np.float64).reshape(np.shape(x))
 
 
 def tree_sum32(v) -> np.float32:

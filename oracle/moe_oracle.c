@@ -48,6 +48,7 @@
 
 #define ORACLE_SOFTMAX 0
 #define ORACLE_SIGMOID 1
+#define ORACLE_SQRTSOFTPLUS 2
 
 /* ------------------------------------------------------------------ bits & bf16 */
 
@@ -120,6 +121,68 @@ void oracle_exp_rl_array(const float* in, float* out, int64_t n)
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_exp_rl(in[i]);
 }
 
+/* ------------------------------------------------------------------ sqrtsoftplus */
+/*
+ * The sqrtsoftplus router score, s = sqrt(softplus(l)), named beside sigmoid in SpecForge
+ * PR #1003 (the load-balance commit: scores are L1-normalised so that sigmoid and
+ * sqrtsoftplus routers share the aux formula). The pages give no formula or precision;
+ * the contract here, fp32 with every operation rounded to nearest:
+ *
+ *   softplus(l) = l                      for l > 20 (log1p(e^l) - l < 2^-28 there)
+ *               = log1p_rl(exp_rl(l))    otherwise
+ *   s           = sqrt(softplus(l))      (IEEE square root, correctly rounded)
+ *
+ * log1p_rl(u), u >= 0, is D. Goldberg's formula ("What every computer scientist should
+ * know about floating-point arithmetic", 1991, Theorem 4): v = 1 + u; u when v == 1, else
+ * (u * ln_rl(v)) / (v - 1), where v - 1 is exact.
+ *
+ * ln_rl(v), v >= 1 finite: v = m * 2^k with m in [1, 2) from the bits, halved (k + 1)
+ * when m > fp32(sqrt 2); f = m - 1 (exact); z = f / (2 + f); ln m = 2 atanh z =
+ * 2z + 2 z^3 (1/3 + w/5 + w^2/7 + w^3/9), w = z^2, |z| <= 0.1716 (the next term is below
+ * 2^-28 relative); the polynomial by Horner with fma and coefficients fp32(1/k); then
+ * ln v = k ln2_hi + (k ln2_lo + ln m), the Cody-Waite split of exp_rl.
+ */
+float oracle_ln_rl(float v)
+{
+    uint32_t b = f2u(v);
+    int k = (int)(b >> 23) - 127;
+    float m = u2f((b & 0x7fffffu) | 0x3f800000u);
+    if (m > (float)1.41421356237309504880) { m = m * 0.5f; k += 1; }
+    const float f = m - 1.0f;
+    const float z = f / (2.0f + f);
+    const float w = z * z;
+    float q = fmaf(w, (float)(1.0 / 9.0), (float)(1.0 / 7.0));
+    q = fmaf(w, q, (float)(1.0 / 5.0));
+    q = fmaf(w, q, (float)(1.0 / 3.0));
+    const float zw = z * w;
+    const float lnm = fmaf(2.0f * zw, q, 2.0f * z);
+    const float hi = ln2_hi_const();
+    const float lo = (float)(0.69314718055994530942 - (double)hi);
+    const float kf = (float)k;
+    return fmaf(kf, hi, fmaf(kf, lo, lnm));
+}
+
+float oracle_log1p_rl(float u)
+{
+    const float v = 1.0f + u;
+    if (v == 1.0f) return u;
+    return (u * oracle_ln_rl(v)) / (v - 1.0f);
+}
+
+float oracle_sqrtsoftplus_rl(float l)
+{
+    const float sp = (l > 20.0f) ? l : oracle_log1p_rl(oracle_exp_rl(l));
+    return sqrtf(sp);
+}
+
+void oracle_fn_array(int which, const float* in, float* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = which == 0 ? oracle_ln_rl(in[i])
+               : which == 1 ? oracle_log1p_rl(in[i])
+                            : oracle_sqrtsoftplus_rl(in[i]);
+}
+
 /* ------------------------------------------------------------------ scores */
 /*
  * Softmax denominator: the fixed 32-lane tree of the contract. Lane L first sums the
@@ -140,11 +203,15 @@ float oracle_tree_sum32(const float* v, int n)
 }
 
 /* Scores of one token (FP32 contract). softmax: m = max, e = exp_rl(l - m), S = tree
- * sum, s = e / S. sigmoid: s = 1 / (1 + exp_rl(-l)). */
+ * sum, s = e / S. sigmoid: s = 1 / (1 + exp_rl(-l)). sqrtsoftplus: see above. */
 void oracle_scores_fp32(int E, const float* l, int score_fn, float* s)
 {
     if (score_fn == ORACLE_SIGMOID) {
         for (int e = 0; e < E; ++e) s[e] = 1.0f / (1.0f + oracle_exp_rl(-l[e]));
+        return;
+    }
+    if (score_fn == ORACLE_SQRTSOFTPLUS) {
+        for (int e = 0; e < E; ++e) s[e] = oracle_sqrtsoftplus_rl(l[e]);
         return;
     }
     if (E <= 0) return;
@@ -380,6 +447,14 @@ void oracle_logits64(int T, int H, int E, const uint16_t* x, const uint16_t* wr,
     }
 }
 
+/* sqrt(softplus(x)) in double with libm: softplus = max(x, 0) + log1p(exp(-|x|)) */
+double oracle_sqrtsoftplus64(double x)
+{
+    if (isnan(x)) return x;
+    return sqrt(fmax(x, 0.0) + log1p(exp(-fabs(x))));
+}
+#define sqrtsoftplus64 oracle_sqrtsoftplus64
+
 /* Weights of given routes from double-precision scores of double logits (masked or
  * invalid ids give 0). renorm: w_j = s_j / sum_j s_j * route_scale; else s_j * scale. */
 void oracle_weights64(int T, int E, int K, const double* logits, const int32_t* ids,
@@ -391,6 +466,8 @@ void oracle_weights64(int T, int E, int K, const double* logits, const int32_t* 
         double* s = (double*)malloc(sizeof(double) * (size_t)E);
         if (score_fn == ORACLE_SIGMOID) {
             for (int e = 0; e < E; ++e) s[e] = 1.0 / (1.0 + exp(-l[e]));
+        } else if (score_fn == ORACLE_SQRTSOFTPLUS) {
+            for (int e = 0; e < E; ++e) s[e] = sqrtsoftplus64(l[e]);
         } else {
             double m = -INFINITY, S = 0.0;
             for (int e = 0; e < E; ++e) if (l[e] > m) m = l[e];
@@ -546,6 +623,8 @@ void oracle_router_stats(int T, int E, int K, const float* logits, const int32_t
         double tot = 0.0;
         if (score_fn == ORACLE_SIGMOID) {
             for (int e = 0; e < E; ++e) s[e] = 1.0 / (1.0 + exp(-(double)l[e]));
+        } else if (score_fn == ORACLE_SQRTSOFTPLUS) {
+            for (int e = 0; e < E; ++e) s[e] = sqrtsoftplus64((double)l[e]);
         } else {
             double m = -INFINITY;
             for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = (double)l[e];

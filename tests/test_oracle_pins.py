@@ -165,7 +165,7 @@ def brute_force_topk(choice, K):
     return list(best)
 
 
-@pytest.mark.parametrize("score_fn", [oracle.SOFTMAX, oracle.SIGMOID])
+@pytest.mark.parametrize("score_fn", [oracle.SOFTMAX, oracle.SIGMOID, oracle.SQRTSOFTPLUS])
 def test_route_ids_brute_force(score_fn):
     rng = np.random.default_rng(5 + score_fn)
     cases = []
@@ -184,7 +184,7 @@ def test_route_ids_brute_force(score_fn):
                 elif mode == 3:
                     l[rng.integers(0, E)] = -0.0          # signed zeros
                     l[rng.integers(0, E)] = 0.0
-                elif mode == 4 and score_fn == oracle.SIGMOID:
+                elif mode == 4 and score_fn != oracle.SOFTMAX:
                     l[rng.integers(0, E)] = np.nan        # a NaN logit
                 bias = None
                 if rng.integers(0, 2):
@@ -211,14 +211,18 @@ def test_route_all_equal_logits_gives_lowest_ids_and_uniform_weights():
 def test_route_weights_renorm_and_scale():
     rng = np.random.default_rng(6)
     for score_fn, scale, K, E in ((oracle.SOFTMAX, 1.0, 8, 128),
-                                  (oracle.SIGMOID, 2.5, 6, 256)):
+                                  (oracle.SIGMOID, 2.5, 6, 256),
+                                  (oracle.SQRTSOFTPLUS, 2.5, 6, 256)):
         l = (rng.standard_normal((200, E)) * 2).astype(F32)
         bias = rng.uniform(-0.05, 0.05, E).astype(F32)
         ids, w, st = oracle.route_fp32(l, K, score_fn, True, scale, sel_bias=bias)
         tot = w.astype(np.float64).sum(1)
         assert np.all(np.abs(tot - scale) <= K * scale * 2.0**-23), np.abs(tot - scale).max()
         # weights are the unbiased float64 scores of the chosen ids, renormalised
-        ref_s = softmax64(l) if score_fn == oracle.SOFTMAX else 1 / (1 + np.exp(-l.astype(float)))
+        lf = l.astype(np.float64)
+        ref_s = {oracle.SOFTMAX: lambda: softmax64(l),
+                 oracle.SIGMOID: lambda: 1 / (1 + np.exp(-lf)),
+                 oracle.SQRTSOFTPLUS: lambda: np.sqrt(np.logaddexp(0.0, lf))}[score_fn]()
         sel = np.take_along_axis(ref_s, ids.astype(np.int64), 1)
         ref_w = sel / sel.sum(1, keepdims=True) * scale
         assert np.allclose(w, ref_w, rtol=1e-6, atol=0)
@@ -570,3 +574,76 @@ def test_grouped_route_brute_force(E, K, n_group, topk_group):
     assert np.array_equal(oracle.route_fp32(l, K, oracle.SOFTMAX, True, n_group=1)[0], a)
     assert np.array_equal(oracle.route_fp32(l, K, oracle.SOFTMAX, True, n_group=n_group,
                                             topk_group=n_group)[0], a)
+
+
+# ------------------------------------------------------------------ sqrtsoftplus score
+
+def test_ln_rl_within_2ulp_of_libm():
+    rng = np.random.default_rng(21)
+    v = np.concatenate([
+        np.linspace(1.0, 4.0, 1 << 19, dtype=np.float64),
+        np.exp(rng.uniform(0, np.log(4.9e8), 1 << 19)),
+        2.0 ** np.arange(0, 29),                                   # k ln2 exactly
+        np.nextafter(np.float32(np.sqrt(2)), [0, 3]).astype(np.float64),  # the halving seam
+    ]).astype(F32)
+    got = oracle.ln_rl(v).astype(np.float64)
+    ref = np.log(v.astype(np.float64))
+    err = np.abs(got - ref) / ulp_f32(np.maximum(ref, 1e-30))
+    err[ref == 0] = np.abs(got[ref == 0])
+    assert oracle.ln_rl(np.array([1.0], F32))[0] == 0.0
+    assert err.max() <= 2.0, err.max()
+    assert np.all(np.diff(oracle.ln_rl(np.sort(v)).astype(np.float64)) >= 0)
+
+
+def test_log1p_rl_within_2ulp_of_libm_and_exact_for_tiny():
+    rng = np.random.default_rng(22)
+    u = np.concatenate([np.exp(rng.uniform(np.log(1e-12), np.log(4.85e8), 1 << 19)),
+                        np.linspace(0, 2, 1 << 16)]).astype(F32)
+    got = oracle.log1p_rl(u).astype(np.float64)
+    ref = np.log1p(u.astype(np.float64))
+    nz = ref > 0
+    err = np.abs(got[nz] - ref[nz]) / ulp_f32(ref[nz])
+    # Goldberg's bound: the log's error (<= 2 ulp, above) plus three roundings of half an
+    # ulp (1 + u, the product, the quotient; v - 1 is exact)
+    assert err.max() <= 3.5, err.max()
+    tiny = np.array([0.0, 2.0 ** -30, 1e-9, 2.0 ** -25], F32)   # 1 + u rounds to 1
+    assert np.array_equal(oracle.log1p_rl(tiny), tiny)
+
+
+def test_sqrtsoftplus_within_3ulp_closed_forms_and_specials():
+    rng = np.random.default_rng(23)
+    x = np.concatenate([np.linspace(-87, 40, 1 << 20), rng.normal(0, 3, 1 << 17)]).astype(F32)
+    got = oracle.sqrtsoftplus_rl(x).astype(np.float64)
+    ref = np.sqrt(np.logaddexp(0.0, x.astype(np.float64)))
+    err = np.abs(got - ref) / ulp_f32(ref)
+    # softplus carries exp_rl's 2 ulp (scaled by u / ((1 + u) log1p u) <= 1) and log1p's
+    # 3.5; the square root halves a relative error and rounds once: <= 3 ulp
+    assert err.max() <= 3.0, err.max()
+    # Goldberg's log1p is not monotone at the ulp level (1 + u and v - 1 step while u
+    # moves): on sorted inputs a score may dip by an ulp or two, never more
+    srt = oracle.sqrtsoftplus_rl(np.sort(x)).astype(np.float64)
+    assert np.all(np.diff(srt) >= -2 * ulp_f32(srt[1:]))
+    # the FP64 reference used by the level-2 weights agrees with numpy's form
+    assert np.allclose(oracle.sqrtsoftplus64(x[:2000].astype(np.float64)), ref[:2000],
+                       rtol=1e-15, atol=0)
+    # above the threshold softplus is l itself: squares give exact roots
+    big = np.array([25, 36, 400, 20.25, 1e30], F32)
+    assert np.array_equal(oracle.sqrtsoftplus_rl(big), np.sqrt(big))
+    s0 = oracle.sqrtsoftplus_rl(np.array([0.0, -0.0], F32)).astype(np.float64)
+    assert np.all(np.abs(s0 - np.sqrt(np.log(2.0))) <= ulp_f32(np.sqrt(np.log(2.0))))
+    sp = oracle.sqrtsoftplus_rl(np.array([-87.5, -1e30, -np.inf, np.inf, np.nan], F32))
+    assert np.all(sp[:3] == 0.0) and sp[3] == np.inf and np.isnan(sp[4])
+    assert np.array_equal(oracle.scores_fp32(x[:999], oracle.SQRTSOFTPLUS),
+                          oracle.sqrtsoftplus_rl(x[:999]))
+
+
+def test_router_stats_sqrtsoftplus_l1_normalised():
+    rng = np.random.default_rng(24)
+    T, E, K = 200, 12, 2
+    l = (rng.standard_normal((T, E)) * 2).astype(F32)
+    ids, _, _ = oracle.route_fp32(l, K, oracle.SQRTSOFTPLUS, True)
+    counts, mp, aux = oracle.router_stats(l, ids, oracle.SQRTSOFTPLUS)
+    s = np.sqrt(np.logaddexp(0.0, l.astype(np.float64)))
+    p = s / s.sum(1, keepdims=True)
+    assert np.allclose(mp, p.mean(0), rtol=1e-12) and mp.sum() == pytest.approx(1.0)
+    assert aux == pytest.approx(E * np.sum(counts / T * p.mean(0)), rel=1e-12)
