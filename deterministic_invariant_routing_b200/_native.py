@@ -23,6 +23,7 @@ MOE_ERR_DEVICE = -6
 
 MOE_SOFTMAX = 0
 MOE_SIGMOID = 1
+MOE_SQRTSOFTPLUS = 2
 
 MOE_ST_NAN_TOKENS = 0
 MOE_ST_ZERO_DENOM = 1

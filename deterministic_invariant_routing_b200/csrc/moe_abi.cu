@@ -49,7 +49,9 @@ int check_cfg(const moe_cfg* c)
     if (c->I < 128 || c->I > 16384 || c->I % 128 != 0) return MOE_ERR_SHAPE;
     if (c->I_shared < 0 || c->I_shared > 32768 || c->I_shared % 128 != 0) return MOE_ERR_SHAPE;
     if ((int64_t)c->T * c->K >= ((int64_t)1 << 31)) return MOE_ERR_SHAPE;
-    if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_SHAPE;
+    if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID &&
+        c->score_fn != MOE_SQRTSOFTPLUS)
+        return MOE_ERR_SHAPE;
     if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_SHAPE;
     if (!isfinite(c->route_scale)) return MOE_ERR_SHAPE;
     if (c->n_group < 0 || c->n_group > 32) return MOE_ERR_SHAPE;

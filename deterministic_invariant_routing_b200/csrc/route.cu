@@ -73,10 +73,9 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             const int e = lane + 32 * i;
             s[i] = (e < E) ? row[e] : 0.0f;
         }
-        if (score_fn == MOE_SIGMOID) {
+        if (score_fn != MOE_SOFTMAX) {
 #pragma unroll
-            for (int i = 0; i < NE; ++i)
-                s[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_rl(-s[i])));
+            for (int i = 0; i < NE; ++i) s[i] = elementwise_score(s[i], score_fn);
         } else {
             float m = -INFINITY;
 #pragma unroll

@@ -1,5 +1,6 @@
 // The FP32 routing contract's device arithmetic, shared by the routing kernel (route.cu)
-// and the router GEMM's fused routing epilogue (tc_gemm.cu): exp_rl and the ordered
+// and the router statistics (stats.cu): exp_rl, the sqrtsoftplus score (SpecForge PR
+// #1003 names it beside sigmoid; its fp32 steps are this contract's) and the ordered
 // selection key. ("DSV4 Flash MoE Train-Inference Consistency Roadmap", Problem 1: router
 // softmax and top-k are validated for precision and stability first; tie-breaking is part
 // of the routing record.)
@@ -39,6 +40,56 @@ __device__ __forceinline__ float exp_rl(float x)
     p = __fmaf_rn(p, r, 1.0f);
     const float two_n = __int_as_float((__float2int_rn(n) + 127) << 23);
     return __fmul_rn(p, two_n);
+}
+
+// ln_rl, for v >= 1 finite: v = m 2^k from the bits (m in [1, 2), halved with k + 1 when
+// above sqrt 2), ln m = 2 atanh(z) with z = (m - 1) / (m + 1) as the odd series through
+// z^9 (coefficients 1/3, 1/5, 1/7, 1/9 rounded once, Horner with fused multiply-adds),
+// then k ln 2 added with the two-part ln 2 of exp_rl.
+__device__ __forceinline__ float ln_rl(float v)
+{
+    const double kLn2 = 0.693147180559945309417232121458;
+    const float kHead = __double2float_rn(rint(kLn2 * 4096.0) / 4096.0);
+    const float kTail = __double2float_rn(kLn2 - (double)kHead);
+    const uint32_t b = __float_as_uint(v);
+    int k = (int)(b >> 23) - 127;
+    float m = __uint_as_float((b & 0x7fffffu) | 0x3f800000u);
+    if (m > __double2float_rn(1.414213562373095048801688724)) {
+        m = __fmul_rn(m, 0.5f);
+        k += 1;
+    }
+    const float f = __fsub_rn(m, 1.0f);  // exact (Sterbenz)
+    const float z = __fdiv_rn(f, __fadd_rn(2.0f, f));
+    const float w = __fmul_rn(z, z);
+    float q = __fmaf_rn(w, __double2float_rn(1.0 / 9.0), __double2float_rn(1.0 / 7.0));
+    q = __fmaf_rn(w, q, __double2float_rn(1.0 / 5.0));
+    q = __fmaf_rn(w, q, __double2float_rn(1.0 / 3.0));
+    const float lnm = __fmaf_rn(__fmul_rn(2.0f, __fmul_rn(z, w)), q, __fmul_rn(2.0f, z));
+    const float kf = __int2float_rn(k);
+    return __fmaf_rn(kf, kHead, __fmaf_rn(kf, kTail, lnm));
+}
+
+// log1p_rl, u >= 0: Goldberg's formula u * ln(1 + u) / ((1 + u) - 1), u itself when
+// 1 + u rounds to 1 (the subtraction is exact)
+__device__ __forceinline__ float log1p_rl(float u)
+{
+    const float v = __fadd_rn(1.0f, u);
+    if (v == 1.0f) return u;
+    return __fdiv_rn(__fmul_rn(u, ln_rl(v)), __fsub_rn(v, 1.0f));
+}
+
+// the sqrtsoftplus score: sqrt(softplus(l)), softplus(l) = l above 20, else
+// log1p_rl(exp_rl(l)); IEEE square root
+__device__ __forceinline__ float sqrtsoftplus_rl(float l)
+{
+    return __fsqrt_rn(l > 20.0f ? l : log1p_rl(exp_rl(l)));
+}
+
+// the score of one logit for the elementwise score functions (sigmoid, sqrtsoftplus)
+__device__ __forceinline__ float elementwise_score(float l, int score_fn)
+{
+    if (score_fn == MOE_SIGMOID) return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_rl(-l)));
+    return sqrtsoftplus_rl(l);
 }
 
 // order-preserving 32-bit image of a choice: -0 == +0, NaN below every number

@@ -2,7 +2,7 @@
 // tokens per expert, the mean L1-normalised score per expert and the Switch-style
 // load-balance value  aux = E * sum_e load_e * mean_prob_e  over the kept tokens (K when
 // balanced), where load_e = tokens_per_expert_e / N and p_{t,e} = s_{t,e} / sum_e' s_{t,e'}
-// with s the unbiased scores of the routing contract (softmax or sigmoid).
+// with s the unbiased scores of the routing contract (softmax, sigmoid or sqrtsoftplus).
 //
 // Deterministic without float atomics: block b owns 256 consecutive tokens, warp w of it
 // 32 of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
@@ -45,10 +45,10 @@ __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __re
             const int e = lane + 32 * i;
             s[i] = (e < E) ? row[e] : 0.0f;
         }
-        if (score_fn == MOE_SIGMOID) {
+        if (score_fn != MOE_SOFTMAX) {
 #pragma unroll
             for (int i = 0; i < NE; ++i)
-                if (lane + 32 * i < E) s[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_rl(-s[i])));
+                if (lane + 32 * i < E) s[i] = elementwise_score(s[i], score_fn);
         } else {
             float m = -INFINITY;
 #pragma unroll

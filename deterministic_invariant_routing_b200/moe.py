@@ -21,6 +21,7 @@ from . import _native as N
 
 SOFTMAX = N.MOE_SOFTMAX
 SIGMOID = N.MOE_SIGMOID
+SQRTSOFTPLUS = N.MOE_SQRTSOFTPLUS
 STATUS_NAMES = ("nan_tokens", "zero_denominator", "bad_expert_id", "pipeline_timeout")
 
 

@@ -30,6 +30,7 @@ import torch
 
 SOFTMAX = 0
 SIGMOID = 1
+SQRTSOFTPLUS = 2
 
 
 @dataclasses.dataclass(frozen=True)

@@ -65,6 +65,14 @@ extern "C" {
 /* score functions */
 #define MOE_SOFTMAX 0
 #define MOE_SIGMOID 1
+/*
+ * sqrtsoftplus score, s = sqrt(softplus(l)) (named beside sigmoid in SpecForge PR #1003,
+ * the load-balance commit; the pages give no formula). fp32, every step rounded to
+ * nearest: softplus(l) = l for l > 20, else log1p_rl(exp_rl(l)), where log1p_rl(u) is
+ * Goldberg's u * ln(1 + u) / ((1 + u) - 1) (u when 1 + u == 1) over a Cody-Waite natural
+ * log (odd atanh series through z^9); then the IEEE square root.
+ */
+#define MOE_SQRTSOFTPLUS 2
 
 /* words of the device status array */
 #define MOE_ST_NAN_TOKENS 0     /* tokens with a NaN selection score */
@@ -91,7 +99,7 @@ typedef struct moe_cfg {
     int32_t K;           /* experts per token (top-k) */
     int32_t I;           /* routed expert intermediate size */
     int32_t I_shared;    /* shared (always-on) expert intermediate size, 0 = none */
-    int32_t score_fn;    /* MOE_SOFTMAX or MOE_SIGMOID */
+    int32_t score_fn;    /* MOE_SOFTMAX, MOE_SIGMOID or MOE_SQRTSOFTPLUS */
     int32_t renorm;      /* 1: weights renormalised over the K selected scores */
     float route_scale;   /* weights are multiplied by it (1.0 = unchanged) */
     /*

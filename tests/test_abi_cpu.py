@@ -56,7 +56,7 @@ def cfg(**over):
 
 @pytest.mark.parametrize("over", [dict(H=100), dict(H=64), dict(I=100), dict(E=0),
                                   dict(E=1025), dict(K=0), dict(K=17), dict(K=9, E=8),
-                                  dict(I_shared=100), dict(T=-1), dict(score_fn=2),
+                                  dict(I_shared=100), dict(T=-1), dict(score_fn=3),
                                   dict(T=200_000_000, K=16),
                                   # group-limited selection
                                   dict(n_group=3, topk_group=1), dict(n_group=4, topk_group=0),

@@ -153,6 +153,12 @@ def test_dsv_sigmoid_shape():
     check_layer("dsv_sigmoid", 8192, n_sample=12)
 
 
+def test_dsv_sqrtsoftplus_shape():
+    """The DeepSeek-style layer with sqrtsoftplus scores (level 1 bit-exact routes from the
+    GPU's logits, level 2 outputs against FP64 sqrt(softplus) weights)."""
+    check_layer("dsv_sigmoid", 4096, n_sample=12, score_fn=synthetic.SQRTSOFTPLUS)
+
+
 def test_dsv_sigmoid_group_limited():
     """The DeepSeek-style layer with group-limited selection (8 groups of 32, 4 kept)."""
     r = check_layer("dsv_sigmoid", 4096, n_sample=12, n_group=8, topk_group=4)

@@ -11,7 +11,7 @@ from helpers import DEV, bits
 
 pytestmark = pytest.mark.gpu
 
-SM, SG = moe.SOFTMAX, moe.SIGMOID
+SM, SG, SP = moe.SOFTMAX, moe.SIGMOID, moe.SQRTSOFTPLUS
 
 
 def adversarial_logits(T, E, seed, std=3.0):
@@ -42,6 +42,9 @@ ROUTE_CASES = [
     (33, 3, SG, 0, 1.0, False, 700),
     (1, 1, SM, 1, 1.0, False, 50),
     (100, 7, SM, 1, 0.5, True, 999),
+    (256, 8, SP, 1, 2.5, True, 2048),   # sqrtsoftplus scores
+    (64, 4, SP, 0, 1.0, False, 700),
+    (1024, 16, SP, 1, 1.0, True, 300),
 ]
 
 
@@ -53,6 +56,7 @@ GROUPED_CASES = [
     (96, 4, SG, False, 3, 1, 999),
     (32, 2, SM, True, 32, 2, 300),      # one expert per group
     (160, 6, SG, True, 20, 20, 700),    # every group kept: plain top-K
+    (256, 8, SP, True, 8, 4, 2048),     # sqrtsoftplus, group-limited
 ]
 
 
@@ -238,11 +242,14 @@ def test_route_injected_near_ties_bit_exact(name, T, n_near):
 
 @pytest.mark.parametrize("name,T,keep", [("qwen3_30b_a3b", 4096, None), ("qwen3_30b_a3b", 3001, 0.8),
                                          ("dsv_sigmoid", 2048, 0.9), ("tiny", 64, None),
-                                         ("dspark", 1000, 0.5)])
+                                         ("dspark", 1000, 0.5), ("dsv_sqrtsoftplus", 2048, 0.9)])
 def test_router_stats_against_oracle(name, T, keep):
     """tokens_per_expert exact, mean_prob and the load-balance value within fp32 summation
     error of the FP64 oracle; the same call twice gives the same bits."""
-    s = synthetic.shape(name, T=T)
+    if name == "dsv_sqrtsoftplus":
+        s = synthetic.shape("dsv_sigmoid", T=T, score_fn=synthetic.SQRTSOFTPLUS)
+    else:
+        s = synthetic.shape(name, T=T)
     l = synthetic.random_logits(T, s.E, seed=T + s.E, std=1.5)
     mask = None if keep is None else synthetic.random_mask(T, keep, 21)
     cfg = moe.Config.of(s)
