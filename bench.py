@@ -46,6 +46,8 @@ def parse():
     p.add_argument("--e2e-chunk", type=int, default=8192,
                    help="tokens per chunk of the host-memory call (copies overlap compute)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip timing the order-invariant combine and the router statistics")
     return p.parse_args()
 
 
@@ -234,11 +236,55 @@ def run_reference(a):
 def workload_config(s, n):
     return {"workload": f"{s.name}_T{s.T}", "T_per_gpu": s.T, "H": s.H, "E": s.E, "K": s.K,
             "I": s.I, "I_shared": s.I_shared,
-            "score_fn": "sigmoid" if s.score_fn == 1 else "softmax", "renorm": bool(s.renorm),
+            "score_fn": ("softmax", "sigmoid", "sqrtsoftplus")[s.score_fn],
+            "renorm": bool(s.renorm),
             "route_scale": s.route_scale, "global_tokens": s.T * n,
             "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
             "l2": "inputs larger than L2 (expert weights and per-step intermediates exceed "
                   "126 MB), no flush"}
+
+
+def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, reps=50):
+    """The next-row calls on this step's tensors, each in its own loop of CUDA-event-timed
+    launches: the order-invariant combine (against the rank-order one) and the router
+    statistics. Their inputs come from the stage API once, outside the timing."""
+    w = layer.w
+    offsets, perm_token, dest_row, x_perm = moe.permute(cfg, b["topk_ids"], x=x)
+    y, ys = moe.grouped_ffn(cfg, x, x_perm, perm_token, offsets, w["w13"], w["w2"],
+                            w.get("w13_s"), w.get("w2_s"))
+    del x_perm
+
+    def loop(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ref = moe.combine(cfg, y, b["topk_w"], dest_row, ys)
+    inv = moe.combine(cfg, y, b["topk_w"], dest_row, ys, order_invariant=True)
+    ms_c = loop(lambda: moe.combine(cfg, y, b["topk_w"], dest_row, ys))
+    ms_i = loop(lambda: moe.combine(cfg, y, b["topk_w"], dest_row, ys, order_invariant=True))
+    ms_s = loop(lambda: moe.router_stats(cfg, b["logits"], offsets))
+    T, H, K, E = cfg.T, cfg.H, cfg.K, cfg.E
+    comb_bytes = T * K * H * 2 + T * H * 2 + T * K * 8 + (T * H * 2 if ys is not None else 0)
+    stat_bytes = T * E * 4
+    same = (ref.view(torch.int16) == inv.view(torch.int16)).float().mean().item()
+    return {
+        "combine_invariant": {"ms": ms_i, "rank_order_combine_ms": ms_c,
+                              "achieved_gbs": comb_bytes / (ms_i * 1e-3) / 1e9,
+                              "frac_hbm": comb_bytes / (ms_i * 1e-3) / 1e9 / hbm_gbs,
+                              "algorithmic_bytes": comb_bytes,
+                              "bits_equal_to_rank_order_fraction": same},
+        "router_stats": {"ms": ms_s, "achieved_gbs": stat_bytes / (ms_s * 1e-3) / 1e9,
+                         "frac_hbm": stat_bytes / (ms_s * 1e-3) / 1e9 / hbm_gbs,
+                         "algorithmic_bytes": stat_bytes},
+        "timing": f"CUDA events, {reps} back-to-back launches each, inputs of one bench step",
+    }
 
 
 def main():
@@ -352,6 +398,8 @@ def main():
         "gpu_launches": K * (9 + (2 if s.I_shared else 0)),
         "clocks": clocks,
     }
+    if not a.no_extras:
+        line["extras"] = time_extras(cfg, layer, x, b, moe, torch, pk["hbm_gbs"])
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         d_cpu = {k: (None if v is None else v.cpu()) for k, v in weights.items()}
         d_cpu["x"] = x.cpu()
