@@ -60,6 +60,10 @@ _SIGS = {
     "oracle_exp_rl": (_F, [_F]),
     "oracle_exp_rl_array": (None, [_P, _P, _I64]),
     "oracle_fn_array": (None, [_I, _P, _P, _I64]),
+    "oracle_dot32": (_F, [_I, _P, _P]),
+    "oracle_combine_bwd_fp32": (None, [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "oracle_router_bwd_fp32": (None, [_I, _I, _I, _P, _P, _P, _P, _I, _I, _F, _P]),
+    "oracle_unpermute_fp32": (None, [_I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "oracle_sqrtsoftplus64": (_D, [_D]),
     "oracle_tree_sum32": (_F, [_P, _I]),
     "oracle_scores_fp32": (None, [_I, _P, _I, _P]),
@@ -354,3 +358,60 @@ def router_stats(logits, ids, score_fn: int, mask=None):
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+# ------------------------------------------------------------------ backward (FP32 contract)
+
+def dot32(a, b) -> np.float32:
+    """The contract's fp32 dot product of two bf16 rows (8-element chunks over 32 lanes)."""
+    a = _arr(a, np.uint16).reshape(-1)
+    b = _arr(b, np.uint16).reshape(-1)
+    return np.float32(lib().oracle_dot32(a.size, _ptr(a), _ptr(b)))
+
+
+def combine_bwd_fp32(dout, y, w, dest_row, rows, mask=None, shared=False):
+    """(dw [T,K] fp32, dy [rows,H] bf16 bits, dy_shared [T,H] bf16 bits or None)."""
+    g = _arr(dout, np.uint16)
+    yy = _arr(y, np.uint16)
+    ww = _arr(w, np.float32)
+    d = _arr(dest_row, np.int32)
+    m = _arr(mask, np.uint8)
+    T, H = g.shape
+    K = d.shape[1]
+    dw = np.empty((T, K), np.float32)
+    dy = np.zeros((max(rows, 1), H), np.uint16)
+    dys = np.empty((T, H), np.uint16) if shared else None
+    lib().oracle_combine_bwd_fp32(T, K, H, _ptr(g), _ptr(yy), _ptr(ww), _ptr(d), _ptr(m),
+                                  _ptr(dw), _ptr(dy), _ptr(dys))
+    return dw, dy[:rows], dys
+
+
+def router_bwd_fp32(logits, ids, dw, score_fn: int, renorm: bool, route_scale: float = 1.0,
+                    mask=None):
+    """dlogits [T,E] fp32 of the contract's router backward."""
+    l = _arr(logits, np.float32)
+    i = _arr(ids, np.int32)
+    g = _arr(dw, np.float32)
+    m = _arr(mask, np.uint8)
+    T, E = l.shape
+    K = i.shape[1]
+    out = np.empty((T, E), np.float32)
+    lib().oracle_router_bwd_fp32(T, E, K, _ptr(l), _ptr(i), _ptr(g), _ptr(m), score_fn,
+                                 int(bool(renorm)), float(route_scale), _ptr(out))
+    return out
+
+
+def unpermute_fp32(dx_rows, dest_row, dx_shared=None, dx_router=None, mask=None):
+    """dx [T,H] bf16 bits: the rank-order sum of a token's row gradients, then the shared
+    expert's and the router's terms, rounded once."""
+    r = _arr(dx_rows, np.uint16)
+    d = _arr(dest_row, np.int32)
+    s = _arr(dx_shared, np.uint16)
+    q = _arr(dx_router, np.uint16)
+    m = _arr(mask, np.uint8)
+    T, K = d.shape
+    H = r.shape[1]
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_unpermute_fp32(T, K, H, _ptr(r), _ptr(d), _ptr(s), _ptr(q), _ptr(m),
+                                _ptr(out))
+    return out

@@ -694,3 +694,144 @@ void oracle_combine_invariant(int T, int K, int H, const uint16_t* y, const floa
         }
     }
 }
+
+/* ------------------------------------------------------------------ backward: FP32 contract */
+/*
+ * The backward of the layer (forward + backward is the contract's scope in "DSV4 Flash MoE
+ * Train-Inference Consistency Roadmap", "Why DSV4 Flash MoE Drifts More Easily" and the
+ * DSV4-WS1-2 row of "Follow-Up Issue Buckets"; the pages fix no backward arithmetic). The
+ * reductions whose order decides bits are specified here and reproduced exactly:
+ *
+ * dot32(a, b), a and b bf16 rows of H: lane L (0..31) owns the 8-element chunks c = L, L+32,
+ * ... (elements 8c .. 8c+7) in increasing order and adds each rounded product
+ * fp32(a_h * b_h) to its fp32 sum (from +0); then butterfly levels 16, 8, 4, 2, 1.
+ */
+float oracle_dot32(int H, const uint16_t* a, const uint16_t* b)
+{
+    float lane[32], nxt[32];
+    for (int l = 0; l < 32; ++l) lane[l] = 0.0f;
+    for (int h = 0; h < H; ++h) {
+        const int L = (h >> 3) & 31;
+        const float p = oracle_bf16_to_f32(a[h]) * oracle_bf16_to_f32(b[h]);
+        lane[L] = lane[L] + p;
+    }
+    for (int off = 16; off >= 1; off >>= 1) {
+        for (int l = 0; l < 32; ++l) nxt[l] = lane[l] + lane[l ^ off];
+        memcpy(lane, nxt, sizeof lane);
+    }
+    return lane[0];
+}
+
+/*
+ * Combine backward: for each kept token t and rank j with a row r = dest_row[t,j] >= 0,
+ * dw[t,j] = dot32(dout_t, y_r) and dy_r = bf16_rne(fp32(w[t,j] * dout_t)); dw = 0 where there
+ * is no row; dy_shared_t = dout_t for kept tokens and +0 for masked ones (their output is 0
+ * whatever x is).
+ */
+void oracle_combine_bwd_fp32(int T, int K, int H, const uint16_t* dout, const uint16_t* y,
+                             const float* w, const int32_t* dest_row, const uint8_t* mask,
+                             float* dw, uint16_t* dy, uint16_t* dy_shared)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const uint16_t* g = dout + (int64_t)t * H;
+        const int kept = !(mask && !mask[t]);
+        for (int j = 0; j < K; ++j) {
+            const int64_t a = (int64_t)t * K + j;
+            const int32_t r = dest_row[a];
+            if (!kept || r < 0) { dw[a] = 0.0f; continue; }
+            dw[a] = oracle_dot32(H, g, y + (int64_t)r * H);
+            for (int h = 0; h < H; ++h)
+                dy[(int64_t)r * H + h] = oracle_f32_to_bf16(w[a] * oracle_bf16_to_f32(g[h]));
+        }
+        if (dy_shared)
+            for (int h = 0; h < H; ++h) dy_shared[(int64_t)t * H + h] = kept ? g[h] : 0;
+    }
+}
+
+/*
+ * Router backward, fp32 contract (one token; every operation rounded to nearest):
+ *   s = the contract scores of the logits (recomputed exactly as in routing);
+ *   renorm:    D = rank-order sum of s_{id_j}; q = rank-order sum of fp32(dw_j * s_{id_j});
+ *              ds_{id_j} = ((route_scale * (dw_j - q / D)) / D); all 0 when D == 0;
+ *   no renorm: ds_{id_j} = route_scale * dw_j;  ds = 0 for experts not selected;
+ *   softmax:      r = rank-order sum of fp32(ds_{id_j} * s_{id_j}); dl_e = s_e * (ds_e - r);
+ *   sigmoid:      dl_e = ds_e * (s_e * (1 - s_e));
+ *   sqrtsoftplus: dl_e = ds_e * (sig_e / (2 * s_e)) with sig_e = 1 / (1 + exp_rl(-l_e)),
+ *                 and 0 where ds_e == 0 or s_e == 0;
+ *   masked tokens: dl = 0. Selection (and so the selection bias) has no gradient.
+ */
+void oracle_router_bwd_fp32(int T, int E, int K, const float* logits, const int32_t* ids,
+                            const float* dw, const uint8_t* mask, int score_fn, int renorm,
+                            float route_scale, float* dlogits)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        float* dl = dlogits + (int64_t)t * E;
+        if (mask && !mask[t]) { for (int e = 0; e < E; ++e) dl[e] = 0.0f; continue; }
+        const float* l = logits + (int64_t)t * E;
+        float* s = (float*)malloc(sizeof(float) * (size_t)E);
+        float* ds = (float*)calloc((size_t)E, sizeof(float));
+        oracle_scores_fp32(E, l, score_fn, s);
+        const int32_t* id = ids + (int64_t)t * K;
+        const float* g = dw + (int64_t)t * K;
+        if (renorm) {
+            float D = 0.0f, q = 0.0f;
+            for (int j = 0; j < K; ++j) {
+                if (id[j] < 0 || id[j] >= E) continue;
+                D = D + s[id[j]];
+                q = q + g[j] * s[id[j]];
+            }
+            if (D != 0.0f) {
+                const float qd = q / D;
+                for (int j = 0; j < K; ++j)
+                    if (id[j] >= 0 && id[j] < E) ds[id[j]] = (route_scale * (g[j] - qd)) / D;
+            }
+        } else {
+            for (int j = 0; j < K; ++j)
+                if (id[j] >= 0 && id[j] < E) ds[id[j]] = route_scale * g[j];
+        }
+        if (score_fn == ORACLE_SOFTMAX) {
+            float r = 0.0f;
+            for (int j = 0; j < K; ++j)
+                if (id[j] >= 0 && id[j] < E) r = r + ds[id[j]] * s[id[j]];
+            for (int e = 0; e < E; ++e) dl[e] = s[e] * (ds[e] - r);
+        } else if (score_fn == ORACLE_SIGMOID) {
+            for (int e = 0; e < E; ++e) dl[e] = ds[e] * (s[e] * (1.0f - s[e]));
+        } else {
+            for (int e = 0; e < E; ++e) {
+                if (ds[e] == 0.0f || s[e] == 0.0f) { dl[e] = 0.0f; continue; }
+                const float sig = 1.0f / (1.0f + oracle_exp_rl(-l[e]));
+                dl[e] = ds[e] * (sig / (2.0f * s[e]));
+            }
+        }
+        free(s);
+        free(ds);
+    }
+}
+
+/*
+ * Un-permute sum of the input gradient: dx_t = bf16_rne(acc), acc from +0 adding, in order,
+ * float(dx_rows[dest_row[t,j]]) for j = 0..K-1 (rows >= 0), then float(dx_shared_t), then
+ * float(dx_router_t) (each when given). Masked tokens: dx_t = +0.
+ */
+void oracle_unpermute_fp32(int T, int K, int H, const uint16_t* dx_rows,
+                           const int32_t* dest_row, const uint16_t* dx_shared,
+                           const uint16_t* dx_router, const uint8_t* mask, uint16_t* dx)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        uint16_t* o = dx + (int64_t)t * H;
+        if (mask && !mask[t]) { for (int h = 0; h < H; ++h) o[h] = 0; continue; }
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < K; ++j) {
+                const int32_t r = dest_row[(int64_t)t * K + j];
+                if (r >= 0) acc = acc + oracle_bf16_to_f32(dx_rows[(int64_t)r * H + h]);
+            }
+            if (dx_shared) acc = acc + oracle_bf16_to_f32(dx_shared[(int64_t)t * H + h]);
+            if (dx_router) acc = acc + oracle_bf16_to_f32(dx_router[(int64_t)t * H + h]);
+            o[h] = oracle_f32_to_bf16(acc);
+        }
+    }
+}
