@@ -47,7 +47,10 @@ def parse():
                    help="tokens per chunk of the host-memory call (copies overlap compute)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
-                   help="skip timing the order-invariant combine and the router statistics")
+                   help="skip timing the order-invariant combine, the router statistics and "
+                        "the backward")
+    p.add_argument("--extras-reps", type=int, default=20,
+                   help="timed repetitions of each extra call")
     return p.parse_args()
 
 
@@ -244,10 +247,11 @@ def workload_config(s, n):
                   "126 MB), no flush"}
 
 
-def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, reps=50):
+def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, tflops, reps=20):
     """The next-row calls on this step's tensors, each in its own loop of CUDA-event-timed
-    launches: the order-invariant combine (against the rank-order one) and the router
-    statistics. Their inputs come from the stage API once, outside the timing."""
+    launches: the order-invariant combine (against the rank-order one), the router
+    statistics and the layer's backward. Their inputs come from the stage API once,
+    outside the timing."""
     w = layer.w
     offsets, perm_token, dest_row, x_perm = moe.permute(cfg, b["topk_ids"], x=x)
     y, ys = moe.grouped_ffn(cfg, x, x_perm, perm_token, offsets, w["w13"], w["w2"],
@@ -271,7 +275,26 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, reps=50):
     ms_i = loop(lambda: moe.combine(cfg, y, b["topk_w"], dest_row, ys, order_invariant=True))
     ms_s = loop(lambda: moe.router_stats(cfg, b["logits"], offsets))
     T, H, K, E = cfg.T, cfg.H, cfg.K, cfg.E
-    comb_bytes = T * K * H * 2 + T * H * 2 + T * K * 8 + (T * H * 2 if ys is not None else 0)
+
+    # backward of the whole layer (moe_backward), dout synthetic
+    from deterministic_invariant_routing_b200 import synthetic
+    has_shared = ys is not None
+    del y, ys
+    dout = synthetic.normal_bf16(T, H, 1.0, 4242, "fill", device=x.device)
+    ws = torch.empty(moe.workspace_bytes(cfg, moe.N.MOE_STAGE_BACKWARD), dtype=torch.uint8,
+                     device=x.device)
+    bwd = lambda: moe.backward(cfg, x, w["w_router"], w["w13"], w["w2"], b["logits"],  # noqa: E731
+                               b["topk_ids"], b["topk_w"], dout, w13_s=w.get("w13_s"),
+                               w2_s=w.get("w2_s"), ws=ws, check=False)
+    ms_b = loop(bwd)
+    rows = int(offsets[-1].item())
+    I, Is = cfg.I, cfg.I_shared
+    # algorithmic: dh, dx rows, dW2, dW13 (12 H I per routed row), router dx and dW, shared
+    bwd_flops = 12 * H * I * rows + 4 * T * H * E + 12 * T * H * Is
+    # executed on top: the recomputed gate_up (twice) and down
+    recompute_flops = 10 * H * I * rows + 6 * T * H * Is
+    del ws
+    comb_bytes = T * K * H * 2 + T * H * 2 + T * K * 8 + (T * H * 2 if has_shared else 0)
     stat_bytes = T * E * 4
     same = (ref.view(torch.int16) == inv.view(torch.int16)).float().mean().item()
     return {
@@ -283,6 +306,13 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, reps=50):
         "router_stats": {"ms": ms_s, "achieved_gbs": stat_bytes / (ms_s * 1e-3) / 1e9,
                          "frac_hbm": stat_bytes / (ms_s * 1e-3) / 1e9 / hbm_gbs,
                          "algorithmic_bytes": stat_bytes},
+        "backward": {"ms": ms_b, "tokens_per_s": T / (ms_b * 1e-3),
+                     "algorithmic_flops": bwd_flops,
+                     "achieved_tflops": bwd_flops / (ms_b * 1e-3) / 1e12,
+                     "frac_bf16_sustained": bwd_flops / (ms_b * 1e-3) / 1e12 / tflops,
+                     "executed_flops_with_recompute": bwd_flops + recompute_flops,
+                     "call": "moe_backward (dx, dW13, dW2, dW_router; forward intermediates "
+                             "recomputed)"},
         "timing": f"CUDA events, {reps} back-to-back launches each, inputs of one bench step",
     }
 
@@ -399,7 +429,8 @@ def main():
         "clocks": clocks,
     }
     if not a.no_extras:
-        line["extras"] = time_extras(cfg, layer, x, b, moe, torch, pk["hbm_gbs"])
+        line["extras"] = time_extras(cfg, layer, x, b, moe, torch, pk["hbm_gbs"],
+                                     pk["bf16_tflops_sustained"], reps=a.extras_reps)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         d_cpu = {k: (None if v is None else v.cpu()) for k, v in weights.items()}
         d_cpu["x"] = x.cpu()

@@ -37,6 +37,7 @@ MOE_STAGE_FFN = 2
 MOE_STAGE_COMBINE = 3
 MOE_STAGE_FORWARD = 4
 MOE_STAGE_STATS = 5
+MOE_STAGE_BACKWARD = 6
 MOE_NUM_STAGE_EVENTS = 8
 
 
@@ -64,6 +65,7 @@ SIGNATURES = {
     "moe_forward": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          _SZ, _P, _P]),
     "moe_router_stats": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_backward": (_I, [_CFG] + [_P] * 21 + [_SZ, _P]),
     "moe_forward_host_workspace_bytes": (_SZ, [_CFG, _I]),
     "moe_forward_host": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),

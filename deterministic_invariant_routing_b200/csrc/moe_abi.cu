@@ -198,6 +198,77 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     return launch_tc_gemm_pair(p, st);
 }
 
+// a grouped bf16 product: out[r] = a_r . B_g^T, B_g = b[g] of [n, k]
+cudaError_t gemm_bf16(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                      int rows, const uint16_t* b, int n, int k, uint16_t* out, int32_t* status,
+                      cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_BF16;
+    p.a = a;
+    p.a_rows = a_rows;
+    p.a_rows_total = a_rows;
+    p.b = b;
+    p.b_rows_per_group = n;
+    p.k = k;
+    p.n = n;
+    p.groups = groups;
+    p.offsets = offsets;
+    p.rows = rows;
+    p.out = out;
+    p.ldo = n;
+    p.status = status;
+    return launch_tc_gemm_pair(p, st);
+}
+
+// the gate/up product recomputed with the SwiGLU backward in its epilogue:
+// dgu[r] = [dh * u * silu'(g) | dh * silu(g)] (bf16, 2I columns)
+cudaError_t gemm_swiglu_bwd(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                            int rows, const uint16_t* w13, int H, int I, const uint16_t* dh,
+                            uint16_t* dgu, int32_t* status, cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_SWIGLU_BWD;
+    p.a = a;
+    p.a_rows = a_rows;
+    p.a_rows_total = a_rows;
+    p.b = w13;
+    p.b_rows_per_group = 2 * I;
+    p.k = H;
+    p.n = I;
+    p.groups = groups;
+    p.offsets = offsets;
+    p.rows = rows;
+    p.out = dgu;
+    p.ldo = 2 * I;
+    p.aux = dh;
+    p.ld_aux = I;
+    p.status = status;
+    return launch_tc_gemm_pair(p, st);
+}
+
+// weight gradient of each group: out[g] [m, n] = sum over the group's K columns of
+// a[m, k] b[n, k] (fp32); a [m, kcols], b [n, kcols], K ranges k_offsets (multiples of 64)
+cudaError_t gemm_wgrad(const uint16_t* a, int m, const uint16_t* b, int n, int64_t kcols,
+                       const int32_t* k_offsets, int groups, float* out, int32_t* status,
+                       cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_WGRAD;
+    p.a = a;
+    p.a_rows = m;
+    p.b = b;
+    p.k = (int)kcols;
+    p.n = n;
+    p.groups = groups;
+    p.rows = m;
+    p.out = out;
+    p.ldo = n;
+    p.k_offsets = k_offsets;
+    p.status = status;
+    return launch_tc_gemm_pair(p, st);
+}
+
 int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm,
              const int32_t* perm_token, const int32_t* offsets,
              const uint16_t* w13, const uint16_t* w2, const uint16_t* w13_s, const uint16_t* w2_s,
@@ -337,6 +408,205 @@ cudaError_t host_pipe(HostPipe** out)
     return cudaSuccess;
 }
 
+size_t pad64(size_t v) { return (v + 63) / 64 * 64; }
+
+// scratch of moe_backward
+struct BwdLayout {
+    size_t offsets, perm_token, dest_row, perm_ws, x_perm, h, y, dy, dh, dgu, dx_perm, w2t, w13t,
+        wrt, poffE, dw_tk, dl, dl_bf, dx_r, poff, colmap, dyT, hT, dguT, xpT, poffT, dlT, xT,
+        h_s, dh_s, dgu_s, dx_s, dy_s, w2st, w13st, dysT, hsT, dgusT, total;
+    int64_t rp, tp, e_pad;
+};
+
+BwdLayout bwd_layout(const moe_cfg& c)
+{
+    BwdLayout L{};
+    const size_t A = (size_t)c.T * c.K, H = c.H, I = c.I, Is = c.I_shared, T = c.T;
+    L.e_pad = (int64_t)pad64(c.E);
+    L.tp = (int64_t)pad64(T > 0 ? T : 1);
+    L.rp = (int64_t)pad64(A + (size_t)63 * c.E);
+    const size_t rp = (size_t)L.rp, tp = (size_t)L.tp, ep = (size_t)L.e_pad;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    L.offsets = take((c.E + 1) * 4);
+    L.perm_token = take(A * 4);
+    L.dest_row = take(A * 4);
+    L.perm_ws = take(permute_ws_bytes(c));
+    L.x_perm = take(A * H * 2);
+    L.h = take(A * I * 2);
+    L.y = take(A * H * 2);
+    L.dy = take(A * H * 2);
+    L.dh = take(A * I * 2);
+    L.dgu = take(A * 2 * I * 2);
+    L.dx_perm = take(A * H * 2);
+    L.w2t = take((size_t)c.E * I * H * 2);
+    L.w13t = take((size_t)c.E * H * 2 * I * 2);
+    L.wrt = take(H * ep * 2);
+    L.poffE = take(2 * 4);
+    L.dw_tk = take(A * 4);
+    L.dl = take(T * c.E * 4);
+    L.dl_bf = take(T * ep * 2);
+    L.dx_r = take(T * H * 2);
+    L.poff = take((c.E + 1) * 4);
+    L.colmap = take(A * 4);
+    L.dyT = take(H * rp * 2);
+    L.hT = take(I * rp * 2);
+    L.dguT = take(2 * I * rp * 2);
+    L.xpT = take(H * rp * 2);
+    L.poffT = take(2 * 4);
+    L.dlT = take(ep * tp * 2);
+    L.xT = take(H * tp * 2);
+    L.h_s = take(T * Is * 2);
+    L.dh_s = take(T * Is * 2);
+    L.dgu_s = take(T * 2 * Is * 2);
+    L.dx_s = take(Is ? T * H * 2 : 0);
+    L.dy_s = take(Is ? T * H * 2 : 0);
+    L.w2st = take(Is * H * 2);
+    L.w13st = take(H * 2 * Is * 2);
+    L.dysT = take(Is ? H * tp * 2 : 0);
+    L.hsT = take(Is * tp * 2);
+    L.dgusT = take(2 * Is * tp * 2);
+    L.total = off;
+    return L;
+}
+
+#define MOE_TRY(call)                                   \
+    do {                                                \
+        const int rc_ = cuda_rc(call);                  \
+        if (rc_ != MOE_OK) return rc_;                  \
+    } while (0)
+
+int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const uint8_t* mask,
+                  const uint16_t* w13, const uint16_t* w2, const uint16_t* w13s,
+                  const uint16_t* w2s, const float* logits, const int32_t* ids,
+                  const float* topk_w, const uint16_t* dout, uint16_t* dx, float* dwr,
+                  float* dw13, float* dw2, float* dw13s, float* dw2s, float* d_topk_w,
+                  float* dlogits, int32_t* status, void* ws, cudaStream_t st)
+{
+    const BwdLayout L = bwd_layout(c);
+    const int64_t A = (int64_t)c.T * c.K;
+    const int H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
+    const int ep = (int)L.e_pad;
+    const bool shared = Is > 0;
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* dest_row = at<int32_t>(ws, L.dest_row);
+    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+    uint16_t* h = at<uint16_t>(ws, L.h);
+    uint16_t* y = at<uint16_t>(ws, L.y);
+    uint16_t* dy = at<uint16_t>(ws, L.dy);
+    uint16_t* dh = at<uint16_t>(ws, L.dh);
+    uint16_t* dgu = at<uint16_t>(ws, L.dgu);
+    uint16_t* dx_perm = at<uint16_t>(ws, L.dx_perm);
+    uint16_t* w2t = at<uint16_t>(ws, L.w2t);
+    uint16_t* w13t = at<uint16_t>(ws, L.w13t);
+    uint16_t* wrt = at<uint16_t>(ws, L.wrt);
+    int32_t* poffE = at<int32_t>(ws, L.poffE);
+    float* dw_tk = d_topk_w ? d_topk_w : at<float>(ws, L.dw_tk);
+    float* dl = dlogits ? dlogits : at<float>(ws, L.dl);
+    uint16_t* dl_bf = at<uint16_t>(ws, L.dl_bf);
+    uint16_t* dx_r = at<uint16_t>(ws, L.dx_r);
+    int32_t* poff = at<int32_t>(ws, L.poff);
+    int32_t* colmap = at<int32_t>(ws, L.colmap);
+    uint16_t* dyT = at<uint16_t>(ws, L.dyT);
+    uint16_t* hT = at<uint16_t>(ws, L.hT);
+    uint16_t* dguT = at<uint16_t>(ws, L.dguT);
+    uint16_t* xpT = at<uint16_t>(ws, L.xpT);
+    int32_t* poffT = at<int32_t>(ws, L.poffT);
+    uint16_t* dlT = at<uint16_t>(ws, L.dlT);
+    uint16_t* xT = at<uint16_t>(ws, L.xT);
+    const int64_t rp = L.rp, tp = L.tp;
+
+    // dispatch and the forward intermediates, recomputed (same kernels, same bits)
+    MOE_TRY(launch_permute(c, ids, offsets, at<int32_t>(ws, L.perm_token), dest_row, status,
+                           at<void>(ws, L.perm_ws), st));
+    MOE_TRY(launch_gather_rows(c, x, dest_row, x_perm, st));
+    MOE_TRY(gate_up(x_perm, A, nullptr, A, offsets, E, 0, w13, H, I, h, status, st));
+    MOE_TRY(down(h, A, offsets, E, 0, w2, H, I, y, status, st));
+
+    // combine backward: routing-weight gradients and the expert-output gradients
+    uint16_t* dy_s = shared ? at<uint16_t>(ws, L.dy_s) : nullptr;
+    MOE_TRY(launch_combine_bwd(c, dout, y, topk_w, dest_row, mask, dw_tk, dy, dy_s, st));
+
+    // routed experts: dh = dy . W2, dgu (SwiGLU backward on the recomputed gate/up
+    // product), dx rows = dgu . W13; the weights as K-major operands ([I,H] and [H,2I])
+    MOE_TRY(launch_transpose(w2, H, I, I, (int64_t)H * I, w2t, H, (int64_t)I * H, E, nullptr, st));
+    MOE_TRY(launch_transpose(w13, 2 * I, H, H, (int64_t)2 * I * H, w13t, 2 * I,
+                             (int64_t)H * 2 * I, E, nullptr, st));
+    MOE_TRY(gemm_bf16(dy, A, offsets, E, 0, w2t, I, H, dh, status, st));
+    MOE_TRY(gemm_swiglu_bwd(x_perm, A, offsets, E, 0, w13, H, I, dh, dgu, status, st));
+    MOE_TRY(gemm_bf16(dgu, A, offsets, E, 0, w13t, H, 2 * I, dx_perm, status, st));
+
+    // router: dlogits, then dx_router = bf16(dlogits) . W_router
+    MOE_TRY(launch_router_bwd(c, logits, ids, dw_tk, mask, dl, dl_bf, ep, st));
+    MOE_TRY(launch_padded_offsets(nullptr, 1, E, poffE, st));
+    MOE_TRY(launch_transpose(wr, E, H, H, 0, wrt, ep, 0, 1, nullptr, st));
+    MOE_TRY(launch_zero_pad(wrt, H, ep, nullptr, poffE, 1, E, st));
+    MOE_TRY(gemm_bf16(dl_bf, T, nullptr, 1, T, wrt, H, ep, dx_r, status, st));
+
+    // shared expert (all kept tokens, dy_shared = dout)
+    uint16_t *h_s = nullptr, *dgu_s = nullptr, *dx_s = nullptr;
+    if (shared) {
+        h_s = at<uint16_t>(ws, L.h_s);
+        uint16_t* dh_s = at<uint16_t>(ws, L.dh_s);
+        dgu_s = at<uint16_t>(ws, L.dgu_s);
+        dx_s = at<uint16_t>(ws, L.dx_s);
+        uint16_t* w2st = at<uint16_t>(ws, L.w2st);
+        uint16_t* w13st = at<uint16_t>(ws, L.w13st);
+        MOE_TRY(gate_up(x, T, nullptr, T, nullptr, 1, T, w13s, H, Is, h_s, status, st));
+        MOE_TRY(launch_transpose(w2s, H, Is, Is, 0, w2st, H, 0, 1, nullptr, st));
+        MOE_TRY(launch_transpose(w13s, 2 * Is, H, H, 0, w13st, 2 * Is, 0, 1, nullptr, st));
+        MOE_TRY(gemm_bf16(dy_s, T, nullptr, 1, T, w2st, Is, H, dh_s, status, st));
+        MOE_TRY(gemm_swiglu_bwd(x, T, nullptr, 1, T, w13s, H, Is, dh_s, dgu_s, status, st));
+        MOE_TRY(gemm_bf16(dgu_s, T, nullptr, 1, T, w13st, H, 2 * Is, dx_s, status, st));
+    }
+
+    // input gradient
+    MOE_TRY(launch_unpermute(c, dx_perm, dest_row, dx_s, dx_r, mask, dx, st));
+
+    // weight gradients: each expert's rows as a K range padded to 64 (zero columns)
+    MOE_TRY(launch_padded_offsets(offsets, E, 0, poff, st));
+    MOE_TRY(launch_colmap(offsets, poff, E, A, colmap, st));
+    MOE_TRY(launch_transpose(dy, A, H, H, 0, dyT, rp, 0, 1, colmap, st));
+    MOE_TRY(launch_zero_pad(dyT, H, rp, offsets, poff, E, 0, st));
+    MOE_TRY(launch_transpose(h, A, I, I, 0, hT, rp, 0, 1, colmap, st));
+    MOE_TRY(launch_zero_pad(hT, I, rp, offsets, poff, E, 0, st));
+    MOE_TRY(launch_transpose(dgu, A, 2 * I, 2 * I, 0, dguT, rp, 0, 1, colmap, st));
+    MOE_TRY(launch_zero_pad(dguT, 2 * I, rp, offsets, poff, E, 0, st));
+    MOE_TRY(launch_transpose(x_perm, A, H, H, 0, xpT, rp, 0, 1, colmap, st));
+    MOE_TRY(launch_zero_pad(xpT, H, rp, offsets, poff, E, 0, st));
+    MOE_TRY(gemm_wgrad(dyT, H, hT, I, rp, poff, E, dw2, status, st));
+    MOE_TRY(gemm_wgrad(dguT, 2 * I, xpT, H, rp, poff, E, dw13, status, st));
+
+    // router weights: dW_router = sum_t bf16(dlogits_t)^T x_t
+    MOE_TRY(launch_padded_offsets(nullptr, 1, T, poffT, st));
+    MOE_TRY(launch_transpose(dl_bf, T, ep, ep, 0, dlT, tp, 0, 1, nullptr, st));
+    MOE_TRY(launch_zero_pad(dlT, ep, tp, nullptr, poffT, 1, T, st));
+    MOE_TRY(launch_transpose(x, T, H, H, 0, xT, tp, 0, 1, nullptr, st));
+    MOE_TRY(launch_zero_pad(xT, H, tp, nullptr, poffT, 1, T, st));
+    MOE_TRY(gemm_wgrad(dlT, E, xT, H, tp, poffT, 1, dwr, status, st));
+
+    if (shared) {
+        uint16_t* dysT = at<uint16_t>(ws, L.dysT);
+        uint16_t* hsT = at<uint16_t>(ws, L.hsT);
+        uint16_t* dgusT = at<uint16_t>(ws, L.dgusT);
+        MOE_TRY(launch_transpose(dy_s, T, H, H, 0, dysT, tp, 0, 1, nullptr, st));
+        MOE_TRY(launch_zero_pad(dysT, H, tp, nullptr, poffT, 1, T, st));
+        MOE_TRY(launch_transpose(h_s, T, Is, Is, 0, hsT, tp, 0, 1, nullptr, st));
+        MOE_TRY(launch_zero_pad(hsT, Is, tp, nullptr, poffT, 1, T, st));
+        MOE_TRY(launch_transpose(dgu_s, T, 2 * Is, 2 * Is, 0, dgusT, tp, 0, 1, nullptr, st));
+        MOE_TRY(launch_zero_pad(dgusT, 2 * Is, tp, nullptr, poffT, 1, T, st));
+        MOE_TRY(gemm_wgrad(dysT, H, hsT, Is, tp, poffT, 1, dw2s, status, st));
+        MOE_TRY(gemm_wgrad(dgusT, 2 * Is, xT, H, tp, poffT, 1, dw13s, status, st));
+    }
+    return MOE_OK;
+}
+
+#undef MOE_TRY
+
 }  // namespace
 }  // namespace moe
 
@@ -344,7 +614,7 @@ using namespace moe;
 
 extern "C" {
 
-MOE_API int moe_abi_version(void) { return 101; }
+MOE_API int moe_abi_version(void) { return 102; }
 
 MOE_API const char* moe_status_string(int code)
 {
@@ -370,6 +640,7 @@ MOE_API size_t moe_workspace_bytes(const moe_cfg* cfg, int stage)
         case MOE_STAGE_COMBINE: return 0;
         case MOE_STAGE_FORWARD: return fwd_layout(*cfg).total;
         case MOE_STAGE_STATS: return stats_ws_bytes(*cfg);
+        case MOE_STAGE_BACKWARD: return bwd_layout(*cfg).total;
         default: return 0;
     }
 }
@@ -604,6 +875,56 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
     // the caller's stream completes only after the last result reached the host
     if ((rc = cuda_rc(cudaEventRecord(hp->done, hp->out))) != MOE_OK) return rc;
     return cuda_rc(cudaStreamWaitEvent(st, hp->done, 0));
+}
+
+MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                         const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                         const uint16_t* w13_s, const uint16_t* w2_s, const float* logits,
+                         const int32_t* topk_ids, const float* topk_w, const uint16_t* dout,
+                         uint16_t* dx, float* dw_router, float* dw13, float* dw2, float* dw13_s,
+                         float* dw2_s, float* d_topk_w, float* dlogits, int32_t* status,
+                         void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc != MOE_OK) return rc;
+    const moe_cfg& c = *cfg;
+    const void* need[] = {w_router, w13, w2, dw_router, dw13, dw2, status};
+    for (const void* q : need)
+        if (q == nullptr) return MOE_ERR_ARG;
+    const void* per_token[] = {x, logits, topk_ids, topk_w, dout, dx};  // NULL allowed at T == 0
+    if (c.T > 0)
+        for (const void* q : per_token)
+            if (q == nullptr) return MOE_ERR_ARG;
+    const void* aligned[] = {x, w_router, w13, w2, logits, topk_ids, topk_w, dout, dx, dw_router,
+                             dw13, dw2, d_topk_w, dlogits};
+    for (const void* q : aligned)
+        if (q != nullptr && !aligned16(q)) return MOE_ERR_ARG;
+    if (c.I_shared > 0) {
+        if (w13_s == nullptr || w2_s == nullptr || dw13_s == nullptr || dw2_s == nullptr)
+            return MOE_ERR_ARG;
+        if (!aligned16(w13_s) || !aligned16(w2_s) || !aligned16(dw13_s) || !aligned16(dw2_s))
+            return MOE_ERR_ARG;
+    }
+    const BwdLayout L = bwd_layout(c);
+    if (ws == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    if (c.T == 0) {
+        // no tokens: every weight gradient is zero
+        const size_t H = c.H, I = c.I, Is = c.I_shared, E = c.E;
+        if ((rc = cuda_rc(cudaMemsetAsync(dw_router, 0, E * H * 4, st))) != MOE_OK) return rc;
+        if ((rc = cuda_rc(cudaMemsetAsync(dw13, 0, E * 2 * I * H * 4, st))) != MOE_OK) return rc;
+        if ((rc = cuda_rc(cudaMemsetAsync(dw2, 0, E * H * I * 4, st))) != MOE_OK) return rc;
+        if (Is > 0) {
+            if ((rc = cuda_rc(cudaMemsetAsync(dw13_s, 0, 2 * Is * H * 4, st))) != MOE_OK) return rc;
+            if ((rc = cuda_rc(cudaMemsetAsync(dw2_s, 0, H * Is * 4, st))) != MOE_OK) return rc;
+        }
+        return MOE_OK;
+    }
+    return backward_impl(c, x, w_router, token_mask, w13, w2, w13_s, w2_s, logits, topk_ids,
+                         topk_w, dout, dx, dw_router, dw13, dw2, dw13_s, dw2_s, d_topk_w, dlogits,
+                         status, ws, st);
 }
 
 }  // extern "C"

@@ -51,8 +51,34 @@ cudaError_t launch_combine_invariant(const moe_cfg& c, const uint16_t* y, const 
                                      const int32_t* dest_row, const uint16_t* y_shared,
                                      const uint8_t* mask, uint16_t* out, cudaStream_t st);
 
+// backward (backward.cu)
+cudaError_t launch_combine_bwd(const moe_cfg& c, const uint16_t* dout, const uint16_t* y,
+                               const float* w, const int32_t* dest_row, const uint8_t* mask,
+                               float* dw, uint16_t* dy, uint16_t* dy_shared, cudaStream_t st);
+cudaError_t launch_router_bwd(const moe_cfg& c, const float* logits, const int32_t* ids,
+                              const float* dw, const uint8_t* mask, float* dl, uint16_t* dl_bf,
+                              int ld_bf, cudaStream_t st);
+cudaError_t launch_unpermute(const moe_cfg& c, const uint16_t* rows, const int32_t* dest_row,
+                             const uint16_t* shared, const uint16_t* router, const uint8_t* mask,
+                             uint16_t* dx, cudaStream_t st);
+cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* poff,
+                                  cudaStream_t st);
+cudaError_t launch_colmap(const int32_t* off, const int32_t* poff, int G, int64_t rows_bound,
+                          int32_t* col, cudaStream_t st);
+cudaError_t launch_transpose(const uint16_t* in, int64_t R, int F, int64_t ld_in, int64_t in_batch,
+                             uint16_t* out, int64_t ld_out, int64_t out_batch, int batches,
+                             const int32_t* colmap, cudaStream_t st);
+cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t* off,
+                            const int32_t* poff, int G, int rows, cudaStream_t st);
+
 // tensor-core GEMMs (tcgen05 / TMEM / TMA)
-enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1 };
+//   EPI_SWIGLU      out[r, c] = bf16(silu(g) * u) of A . B_g^T (gate and up columns paired)
+//   EPI_BF16        out[r, c] = bf16(A . B_g^T)
+//   EPI_SWIGLU_BWD  the gate/up product recomputed; with dh = aux[r, c] (bf16):
+//                   out[r, c] = bf16(dh * u * silu'(g)), out[r, n + c] = bf16(dh * silu(g))
+//   EPI_WGRAD       grouped over K: out[g][m, c] = fp32(sum over k in [k_offsets[g],
+//                   k_offsets[g+1]) of A[m, k] * B[c, k]) -- an expert's rows contracted
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
 
 struct GemmProblem {
     int epilogue;            // GemmEpilogue
@@ -60,20 +86,23 @@ struct GemmProblem {
     int64_t a_rows;          // rows of the A buffer (TMA bound)
     const int32_t* gather_rows;  // grouped row r reads A row gather_rows[r] (NULL: row r)
     int64_t a_rows_total;    // grouped rows (bound of offsets[groups])
-    const uint16_t* b;       // B [groups * b_rows_per_group, k] bf16
+    const uint16_t* b;       // B [groups * b_rows_per_group, k] bf16 (EPI_WGRAD: [n, k])
     int b_rows_per_group;    // SWIGLU: 2*I (gate rows then up rows); else N
-    int k;                   // reduction length (multiple of 64)
+    int k;                   // reduction length (multiple of 64; EPI_WGRAD: A's and B's width)
     int n;                   // output columns per group (SWIGLU: I)
     int groups;              // number of row groups (experts)
     const int32_t* offsets;  // device [groups+1] row ranges of A, or NULL: one group [0, rows)
-    int rows;                // rows when offsets == NULL
+    int rows;                // rows when offsets == NULL (EPI_WGRAD: rows of A = M)
     void* out;               // output [*, ldo]
     int64_t ldo;             // output row stride in elements
-    const float* bias;       // EPI_F32: per-column bias or NULL
+    const float* bias;       // unused by the pair kernel
     int32_t* status;         // device status words (MOE_ST_PIPE_TIMEOUT) or NULL
+    const uint16_t* aux;     // EPI_SWIGLU_BWD: dh [rows, ld_aux] bf16
+    int64_t ld_aux;
+    const int32_t* k_offsets;  // EPI_WGRAD: device [groups+1] K ranges (multiples of 64)
 };
 
-// the grouped expert products (EPI_SWIGLU / EPI_BF16) on CTA pairs
+// the grouped expert products on CTA pairs
 cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st);
 
 // the router product: logits[T,E] = x . Wr^T (+ logit_bias), fp32

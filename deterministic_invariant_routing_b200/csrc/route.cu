@@ -66,40 +66,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             }
             continue;
         }
-        const float* row = logits + (int64_t)t * E;
         float s[NE];
-#pragma unroll
-        for (int i = 0; i < NE; ++i) {
-            const int e = lane + 32 * i;
-            s[i] = (e < E) ? row[e] : 0.0f;
-        }
-        if (score_fn != MOE_SOFTMAX) {
-#pragma unroll
-            for (int i = 0; i < NE; ++i) s[i] = elementwise_score(s[i], score_fn);
-        } else {
-            float m = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < NE; ++i)
-                if (lane + 32 * i < E && s[i] > m) m = s[i];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-                const float o = __shfl_xor_sync(0xffffffffu, m, off);
-                if (o > m) m = o;
-            }
-            float part = 0.0f;
-#pragma unroll
-            for (int i = 0; i < NE; ++i) {
-                if (lane + 32 * i < E) {
-                    s[i] = exp_rl(__fsub_rn(s[i], m));
-                    part = __fadd_rn(part, s[i]);
-                }
-            }
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
-#pragma unroll
-            for (int i = 0; i < NE; ++i) s[i] = __fdiv_rn(s[i], part);
-        }
+        contract_scores<NE>(logits + (int64_t)t * E, E, score_fn, lane, s);
         // selection keys; empty slots get key 0 (below every real key)
         unsigned long long key[NE];
         bool any_nan = false;

@@ -92,6 +92,49 @@ __device__ __forceinline__ float elementwise_score(float l, int score_fn)
     return sqrtsoftplus_rl(l);
 }
 
+// The contract scores of one token's logits row, one warp: lane L holds experts L, L+32, ...
+// (s[i] for expert L + 32 i; slots past E hold values that are never used). softmax: max
+// by comparisons and a butterfly, e = exp_rl(l - m), the 32-lane tree sum (each lane's
+// experts in increasing order, then butterfly levels 16 .. 1), s = e / S; sigmoid and
+// sqrtsoftplus elementwise.
+template <int NE>
+__device__ __forceinline__ void contract_scores(const float* __restrict__ row, int E,
+                                                int score_fn, int lane, float (&s)[NE])
+{
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+        const int e = lane + 32 * i;
+        s[i] = (e < E) ? row[e] : 0.0f;
+    }
+    if (score_fn != MOE_SOFTMAX) {
+#pragma unroll
+        for (int i = 0; i < NE; ++i) s[i] = elementwise_score(s[i], score_fn);
+        return;
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NE; ++i)
+        if (lane + 32 * i < E && s[i] > m) m = s[i];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, m, off);
+        if (o > m) m = o;
+    }
+    float part = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+        if (lane + 32 * i < E) {
+            s[i] = exp_rl(__fsub_rn(s[i], m));
+            part = __fadd_rn(part, s[i]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
+#pragma unroll
+    for (int i = 0; i < NE; ++i) s[i] = __fdiv_rn(s[i], part);
+}
+
 // order-preserving 32-bit image of a choice: -0 == +0, NaN below every number
 __device__ __forceinline__ uint32_t order_bits(float c)
 {

@@ -59,6 +59,11 @@ struct PairArgs {
     void* out;
     int64_t ldo;
     int32_t* status;
+    int m_tiles;                 // EPI_WGRAD: row tiles of A (per group)
+    const int32_t* k_offsets;    // EPI_WGRAD: [groups+1] K ranges
+    const uint16_t* aux;         // EPI_SWIGLU_BWD: dh
+    int64_t ld_aux;
+    int half_out;                // EPI_SWIGLU_BWD: column of the first up gradient
 };
 
 template <int EPI, int NP>
@@ -81,10 +86,13 @@ struct Cfg2 {
 struct PairTile {
     int g, n;
     int64_t row0, row_end;  // row0: the pair tile's first row
+    int k0, kbs;            // first K column and k-blocks of the tile's reduction
 };
 
+// row-grouped products: tiles of 256 rows inside each group's row range, n fastest
 __device__ __forceinline__ PairTile decode_pair_tile(int t, int n_tiles, int groups,
-                                                     const int32_t* prefix, const int32_t* offs)
+                                                     const int32_t* prefix, const int32_t* offs,
+                                                     int k_blocks)
 {
     PairTile ti;
     const int mt = t / n_tiles;
@@ -98,6 +106,25 @@ __device__ __forceinline__ PairTile decode_pair_tile(int t, int n_tiles, int gro
     ti.g = lo;
     ti.row0 = (int64_t)offs[lo] + (int64_t)(mt - prefix[lo]) * PM;
     ti.row_end = offs[lo + 1];
+    ti.k0 = 0;
+    ti.kbs = k_blocks;
+    return ti;
+}
+
+// K-grouped products (EPI_WGRAD): group g owns K columns [k_offsets[g], k_offsets[g+1]);
+// tiles are (g, row tile, n), n fastest
+__device__ __forceinline__ PairTile decode_wgrad_tile(int t, const PairArgs& a)
+{
+    PairTile ti;
+    const int per = a.m_tiles * a.n_tiles;
+    ti.g = t / per;
+    const int rem = t - ti.g * per;
+    const int mt = rem / a.n_tiles;
+    ti.n = rem - mt * a.n_tiles;
+    ti.row0 = (int64_t)mt * PM;
+    ti.row_end = a.rows;
+    ti.k0 = a.k_offsets[ti.g];
+    ti.kbs = (a.k_offsets[ti.g + 1] - ti.k0) / BK;
     return ti;
 }
 
@@ -183,7 +210,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
     cluster_sync();  // barriers and TMEM of both CTAs ready before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
-    const int total = prefix[G] * args.n_tiles;
+    constexpr bool kWgrad = (EPI == EPI_WGRAD);
+    constexpr bool kGateUp = (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD);
+    const int total = kWgrad ? G * args.m_tiles * args.n_tiles : prefix[G] * args.n_tiles;
+    auto decode = [&](int t) -> PairTile {
+        if (kWgrad) return decode_wgrad_tile(t, args);
+        return decode_pair_tile(t, args.n_tiles, G, prefix, offs, args.k_blocks);
+    };
 
     if (warp == 0 && !GATHER) {
         // -------------------------------------------------------------- TMA producer
@@ -193,23 +226,24 @@ __global__ void __launch_bounds__(kThreads2, 1)
             uint32_t phase = 0;
             uint32_t armed = 0, armed_phase = 0;
             for (int t = cluster; t < total && !*abort_flag; t += nclusters) {
-                const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+                const PairTile ti = decode(t);
                 const int arow = (int)ti.row0 + (int)rank * HM;
-                const int brow = (EPI == EPI_SWIGLU)
-                                     ? ti.g * args.b_rows_per_group +
-                                           (leader ? 0 : args.half_rows) + ti.n * kBRows
-                                     : ti.g * args.b_rows_per_group + ti.n * NP +
-                                           (int)rank * kBRows;
+                const int brow = kGateUp ? ti.g * args.b_rows_per_group +
+                                               (leader ? 0 : args.half_rows) + ti.n * kBRows
+                                 : kWgrad ? ti.n * NP + (int)rank * kBRows
+                                          : ti.g * args.b_rows_per_group + ti.n * NP +
+                                                (int)rank * kBRows;
                 bool ok = true;
-                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                for (int kb = 0; kb < ti.kbs; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = mapa_shared(full_bar(stage), 0);
                     if (leader) mbar_expect_tx(full_bar(stage), 2 * C::kStageBytes);
-                    tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, kb * BK, arow, fb);
-                    tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kb * BK, brow, fb);
+                    const int kx = ti.k0 + kb * BK;
+                    tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, kx, arow, fb);
+                    tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kx, brow, fb);
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) {
@@ -251,12 +285,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
         };
         for (int t = cluster; t < total; t += nclusters) {
             if (!__shfl_sync(0xffffffffu, lane == 0 ? !*abort_flag : 0, 0)) break;
-            const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+            const PairTile ti = decode(t);
             const int arow = (int)ti.row0 + (int)rank * HM;
-            const int brow = (EPI == EPI_SWIGLU)
-                                 ? ti.g * args.b_rows_per_group + (leader ? 0 : args.half_rows) +
-                                       ti.n * kBRows
-                                 : ti.g * args.b_rows_per_group + ti.n * NP + (int)rank * kBRows;
+            const int brow = kGateUp ? ti.g * args.b_rows_per_group +
+                                           (leader ? 0 : args.half_rows) + ti.n * kBRows
+                                     : ti.g * args.b_rows_per_group + ti.n * NP +
+                                           (int)rank * kBRows;
             if (GATHER) {
                 // source token of each of this CTA's 128 rows; rows past the group's end
                 // repeat its last row (computed, never stored)
@@ -270,7 +304,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 __syncwarp();
             }
             int ok = 1;
-            for (int kb = 0; kb < args.k_blocks; ++kb) {
+            for (int kb = 0; kb < ti.kbs; ++kb) {
                 if (lane == 0)
                     ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -328,8 +362,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NP);
+                const int kbs = decode(t).kbs;
                 bool ok = true;
-                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                for (int kb = 0; kb < kbs; ++kb) {
                     if (!wait_bounded(full_bar(stage), phase, abort_flag, args.status)) {
                         ok = false;
                         break;
@@ -394,7 +429,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         };
         int i = 0;
         for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
-            const PairTile ti = decode_pair_tile(t, args.n_tiles, G, prefix, offs);
+            const PairTile ti = decode(t);
             const int acc = i & 1;
             int ok = 1;
             if (lane == 0)
@@ -429,6 +464,73 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     const int col = ti.n * (NP / 2) + c;
                     store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
                 }
+            } else if (EPI == EPI_SWIGLU_BWD) {
+                // dh of this row's 32 intermediate columns, then the SwiGLU derivatives:
+                // silu(g) = g s, s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s))
+#pragma unroll 1
+                for (int c = 0; c < NP / 2; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(tbase + (uint32_t)c, g);
+                    tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
+                    const int col = ti.n * (NP / 2) + c;
+                    uint32_t dhw[16];
+                    if (valid) {
+                        const uint4* src =
+                            reinterpret_cast<const uint4*>(args.aux + grow * args.ld_aux + col);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const uint4 q4 = src[v];
+                            dhw[4 * v] = q4.x;
+                            dhw[4 * v + 1] = q4.y;
+                            dhw[4 * v + 2] = q4.z;
+                            dhw[4 * v + 3] = q4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) dhw[j] = 0u;
+                    }
+                    uint32_t pg[16], pu[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float dg2[2], du2[2];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const float gv = __uint_as_float(g[2 * j + h2]);
+                            const float uv = __uint_as_float(u[2 * j + h2]);
+                            const float dh = __uint_as_float(h2 ? (dhw[j] & 0xffff0000u)
+                                                                : (dhw[j] << 16));
+                            const float sg = __frcp_rn(1.0f + __expf(-gv));
+                            const float dsilu = sg * (1.0f + gv * (1.0f - sg));
+                            dg2[h2] = dh * uv * dsilu;
+                            du2[h2] = dh * (gv * sg);
+                        }
+                        pg[j] = bf16x2_rne(dg2[0], dg2[1]);
+                        pu[j] = bf16x2_rne(du2[0], du2[1]);
+                    }
+                    store_block(pg, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
+                    const int ucol = args.half_out + col;
+                    store_block(pu, full_blk, valid, row_blk, ucol, out + grow * args.ldo + ucol);
+                }
+            } else if (EPI == EPI_WGRAD) {
+                // fp32 weight gradient rows of group g; a group with no rows gives zeros
+                float* o = static_cast<float*>(args.out);
+#pragma unroll 1
+                for (int c = 0; c < NP; c += 32) {
+                    uint32_t r[32];
+                    if (ti.kbs > 0) {
+                        tmem_ld32(tbase + (uint32_t)c, r);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] = 0u;
+                    }
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            o + ((int64_t)ti.g * args.rows + grow) * args.ldo + ti.n * NP + c);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                    }
+                }
             } else {
 #pragma unroll 1
                 for (int c = 0; c < NP; c += 32) {
@@ -462,7 +564,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
 {
     using C = Cfg2<EPI, NP>;
     auto kernel = tc_gemm_pair_kernel<EPI, NP, GATHER>;
-    const int groups = p.offsets ? p.groups : 1;
+    const int groups = (p.offsets || EPI == EPI_WGRAD) ? p.groups : 1;
     const size_t smem = C::smem_bytes(groups);
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -499,25 +601,40 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     }
     const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
     CUtensorMap ma, mb, mo;
+    const bool wgrad = (EPI == EPI_WGRAD);
     if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) return cudaErrorInvalidValue;
-    if (!make_map(&mb, p.b, (int64_t)groups * p.b_rows_per_group, p.k, NP / 2))
+    if (!make_map(&mb, p.b, wgrad ? (int64_t)p.n : (int64_t)groups * p.b_rows_per_group, p.k,
+                  NP / 2))
         return cudaErrorInvalidValue;
-    if (!make_store_map(&mo, p.out, rows_total, p.n, p.ldo)) return cudaErrorInvalidValue;
+    if (wgrad) {
+        mo = mb;  // fp32 rows are stored from registers; the store map is not used
+    } else {
+        const int out_cols = (EPI == EPI_SWIGLU_BWD) ? 2 * p.n : p.n;
+        if (!make_store_map(&mo, p.out, rows_total, out_cols, p.ldo))
+            return cudaErrorInvalidValue;
+    }
     PairArgs a;
     a.k_blocks = p.k / BK;
-    a.n_tiles = (EPI == EPI_SWIGLU) ? p.n / (NP / 2) : p.n / NP;
+    constexpr bool kGateUpL = (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD);
+    a.n_tiles = kGateUpL ? p.n / (NP / 2) : p.n / NP;
     a.groups = groups;
     a.offsets = p.offsets;
     a.rows = p.rows;
     a.b_rows_per_group = p.b_rows_per_group;
-    a.half_rows = (EPI == EPI_SWIGLU) ? p.n : 0;
+    a.half_rows = kGateUpL ? p.n : 0;
+    a.m_tiles = wgrad ? (int)((p.rows + PM - 1) / PM) : 0;
+    a.k_offsets = p.k_offsets;
+    a.aux = p.aux;
+    a.ld_aux = p.ld_aux;
+    a.half_out = (EPI == EPI_SWIGLU_BWD) ? p.n : 0;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;
     a.out = p.out;
     a.ldo = p.ldo;
     a.status = p.status;
-    const int64_t max_tiles = ((rows_total + PM - 1) / PM + groups) * a.n_tiles;
+    const int64_t max_tiles = wgrad ? (int64_t)groups * a.m_tiles * a.n_tiles
+                                    : ((rows_total + PM - 1) / PM + groups) * a.n_tiles;
     int64_t clusters = max_clusters[dev];
     if (max_tiles < clusters) clusters = max_tiles;
     if (clusters < 1) clusters = 1;
@@ -536,6 +653,16 @@ cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st)
         return launch_pair_variant<EPI_SWIGLU, 256, false>(p, st);
     }
     if (p.gather_rows) return cudaErrorInvalidValue;
+    if (p.epilogue == EPI_SWIGLU_BWD) {
+        if (p.n % 128 != 0 || p.aux == nullptr) return cudaErrorInvalidValue;
+        return launch_pair_variant<EPI_SWIGLU_BWD, 256, false>(p, st);
+    }
+    if (p.epilogue == EPI_WGRAD) {
+        if (p.k_offsets == nullptr || p.rows < 1) return cudaErrorInvalidValue;
+        if (p.n % 256 == 0) return launch_pair_variant<EPI_WGRAD, 256, false>(p, st);
+        if (p.n % 128 == 0) return launch_pair_variant<EPI_WGRAD, 128, false>(p, st);
+        return cudaErrorInvalidValue;
+    }
     if (p.epilogue == EPI_BF16) {
         if (p.n % 256 == 0) return launch_pair_variant<EPI_BF16, 256, false>(p, st);
         if (p.n % 128 == 0) return launch_pair_variant<EPI_BF16, 128, false>(p, st);

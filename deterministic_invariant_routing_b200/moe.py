@@ -240,6 +240,52 @@ def router_stats(cfg: Config, logits, offsets, token_mask=None):
     return {"tokens_per_expert": counts, "mean_prob": mp, "aux": aux}
 
 
+# ------------------------------------------------------------------ backward
+
+def backward(cfg: Config, x, w_router, w13, w2, logits, topk_ids, topk_w, dout, token_mask=None,
+             w13_s=None, w2_s=None, ws=None, status=None, keep: bool = False,
+             check: bool = True) -> dict:
+    """Gradients of sum(dout * out) of the layer for the forward's routes (moe_backward):
+    {dx [T,H] bf16, dw_router [E,H], dw13 [E,2I,H], dw2 [E,H,I] fp32 (+ dw13_s, dw2_s with a
+    shared expert)}; keep=True adds d_topk_w [T,K] and dlogits [T,E] (fp32).
+    logits, topk_ids, topk_w: as forward(keep=True) returned them."""
+    dev = x.device
+    T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
+    _need(x, "x", torch.bfloat16, (T, H), dev)
+    _need(w_router, "w_router", torch.bfloat16, (E, H), dev)
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H), dev)
+    _need(w2, "w2", torch.bfloat16, (E, H, I), dev)
+    _need(logits, "logits", torch.float32, (T, E), dev)
+    _need(topk_ids, "topk_ids", torch.int32, (T, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (T, K), dev)
+    _need(dout, "dout", torch.bfloat16, (T, H), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    if Is:
+        _need(w13_s, "w13_s", torch.bfloat16, (2 * Is, H), dev)
+        _need(w2_s, "w2_s", torch.bfloat16, (H, Is), dev)
+    g = {"dx": torch.empty(T, H, dtype=torch.bfloat16, device=dev),
+         "dw_router": torch.empty(E, H, dtype=torch.float32, device=dev),
+         "dw13": torch.empty(E, 2 * I, H, dtype=torch.float32, device=dev),
+         "dw2": torch.empty(E, H, I, dtype=torch.float32, device=dev),
+         "dw13_s": torch.empty(2 * Is, H, dtype=torch.float32, device=dev) if Is else None,
+         "dw2_s": torch.empty(H, Is, dtype=torch.float32, device=dev) if Is else None}
+    if keep:
+        g["d_topk_w"] = torch.empty(T, K, dtype=torch.float32, device=dev)
+        g["dlogits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
+    nbytes = workspace_bytes(cfg, N.MOE_STAGE_BACKWARD)
+    ws = _ws(nbytes, dev, ws)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_backward(ctypes.byref(cfg.c()), _p(x), _p(w_router), _p(token_mask),
+                              _p(w13), _p(w2), _p(w13_s), _p(w2_s), _p(logits), _p(topk_ids),
+                              _p(topk_w), _p(dout), _p(g["dx"]), _p(g["dw_router"]),
+                              _p(g["dw13"]), _p(g["dw2"]), _p(g["dw13_s"]), _p(g["dw2_s"]),
+                              _p(g.get("d_topk_w")), _p(g.get("dlogits")), _p(st), _p(ws),
+                              nbytes, _stream(dev)), "moe_backward")
+    if check:
+        check_status(st)
+    return g
+
+
 # ------------------------------------------------------------------ whole layer
 
 def forward(cfg: Config, x, w_router, w13, w2, logit_bias=None, sel_bias=None, token_mask=None,

@@ -88,6 +88,7 @@ extern "C" {
 #define MOE_STAGE_COMBINE 3
 #define MOE_STAGE_FORWARD 4
 #define MOE_STAGE_STATS 5
+#define MOE_STAGE_BACKWARD 6
 
 /* number of CUDA events moe_forward can record (stage boundaries), see moe_forward */
 #define MOE_NUM_STAGE_EVENTS 8
@@ -316,6 +317,43 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
                              const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out_host,
                              int32_t* status, int chunk_tokens, void* ws, size_t ws_bytes,
                              void* stream);
+
+/*
+ * Backward of the whole layer (forward + backward is the contract's scope: "DSV4 Flash MoE
+ * Train-Inference Consistency Roadmap", "Why DSV4 Flash MoE Drifts More Easily" and the
+ * DSV4-WS1-2 row of "Follow-Up Issue Buckets"; the pages give no backward arithmetic).
+ * Gradients of sum(dout * out) for the routes of the forward (selection has no gradient).
+ * The forward intermediates are recomputed from x with the forward's kernels (same bits).
+ *
+ *  Inputs (DEVICE): x, w_router, token_mask (or NULL), w13, w2, w13_s/w2_s as in
+ *    moe_forward; logits [T,E] fp32, topk_ids [T,K], topk_w [T,K] as the forward returned
+ *    them; dout [T,H] bf16.
+ *  Outputs (DEVICE, written completely):
+ *    dx [T,H] bf16, dw_router [E,H] fp32, dw13 [E,2I,H] fp32, dw2 [E,H,I] fp32,
+ *    dw13_s [2I_shared,H] / dw2_s [H,I_shared] fp32 (required when I_shared > 0),
+ *    d_topk_w [T,K] fp32 and dlogits [T,E] fp32 (optional boundary outputs, NULL = not kept).
+ *  Arithmetic (fixed order, no float atomics: bitwise repeatable; dx of a token depends
+ *  only on its own row):
+ *    d_topk_w[t,j] = dot32(dout_t, y_row): lane L of 32 sums the rounded products of the
+ *      8-element chunks L, L+32, ... in order, then butterfly levels 16..1 (fp32);
+ *    dy_row = bf16(topk_w[t,j] * dout_t); dy_shared = dout (0 for masked tokens);
+ *    dh = bf16(dy . W2_e); [dg | du] = bf16(dh * u * silu'(g) | dh * silu(g)) with g, u the
+ *      recomputed fp32 gate/up products; dx_row = bf16([dg | du] . W13_e);
+ *    dlogits: through the renormalisation and the score function in fp32, each operation
+ *      rounded to nearest, rank-order sums (see the router backward of the oracle);
+ *    dx_t = bf16(rank-order sum of dx_row + shared term + bf16(dlogits_t) . W_router), +0
+ *      for masked tokens;
+ *    dW = sum over an expert's rows, ascending, of dy^T h / [dg|du]^T x (fp32 accumulation
+ *      on the tensor cores, bf16 operands); dW_router = sum_t bf16(dlogits_t)^T x_t.
+ *  ws  moe_workspace_bytes(cfg, MOE_STAGE_BACKWARD) bytes.
+ */
+MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                         const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                         const uint16_t* w13_s, const uint16_t* w2_s, const float* logits,
+                         const int32_t* topk_ids, const float* topk_w, const uint16_t* dout,
+                         uint16_t* dx, float* dw_router, float* dw13, float* dw2, float* dw13_s,
+                         float* dw2_s, float* d_topk_w, float* dlogits, int32_t* status,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* Text of a return code. */
 MOE_API const char* moe_status_string(int code);
