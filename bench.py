@@ -262,6 +262,10 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, tflops, reps=20):
         for _ in range(3):
             fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # hold the stream while the calls are queued, so that the events time the device's
+        # back-to-back work and not the host's launch rate
+        torch.cuda.synchronize()
+        torch.cuda._sleep(50_000_000)
         e0.record()
         for _ in range(reps):
             fn()

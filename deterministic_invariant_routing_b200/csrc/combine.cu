@@ -115,16 +115,25 @@ cudaError_t launch_k(const moe_cfg& c, const uint16_t* y, const float* w, const 
 // Order-invariant variant ("From Expert Reduction to Behavioral Divergence", arXiv
 // 2607.28097, Abstract: scheme C's result does not depend on the order of the expert
 // terms). Per output element the terms -- w_j * y_j formed exactly in double, and the
-// shared expert's y -- are put in a canonical order (ascending magnitude, the negative of
-// equal magnitudes first) by an odd-even transposition network, summed in double, and
-// rounded once to fp32 then to bf16. The result is a function of the multiset of terms.
-__device__ __forceinline__ bool canon_after(double a, bool va, double b, bool vb)
+// shared expert's y -- are summed in double in a canonical order (ascending magnitude, the
+// negative of equal magnitudes first) and rounded once to fp32 then to bf16, so the result
+// is a function of the multiset of terms.
+//
+// Two routes to the same bits. Every term has at most 32 significant bits (24 x 8), so when
+// the valid nonzero terms' exponents lie within 16 of each other every partial sum of up to
+// 17 of them fits in double's 53 bits exactly: any order gives the exact sum, and the terms
+// are added as they come. Otherwise (or with an infinite / NaN term) they are sorted by the
+// 64-bit key (|x| bits << 1) | (x is not negative) -- ascending magnitude, -x before +x --
+// with an odd-even transposition network on integers, and added in that order.
+__device__ __forceinline__ uint64_t canon_key(double x)
 {
-    // should slot a (valid va) come after slot b? invalid slots go last
-    if (!va) return vb;
-    if (!vb) return false;
-    const double fa = fabs(a), fb = fabs(b);
-    return fa != fb ? fa > fb : a > b;
+    const uint64_t b = (uint64_t)__double_as_longlong(x);
+    return ((b & 0x7fffffffffffffffull) << 1) | ((b >> 63) ^ 1ull);
+}
+
+__device__ __forceinline__ double from_key(uint64_t k)
+{
+    return __longlong_as_double((long long)((k >> 1) | ((~k & 1ull) << 63)));
 }
 
 template <int KMAX>
@@ -156,38 +165,53 @@ __global__ void __launch_bounds__(256) combine_invariant_kernel(
         ok[KMAX] = y_shared != nullptr;
         wj[KMAX] = 1.0f;
         rows[KMAX] = ok[KMAX] ? y_shared[idx] : make_uint4(0u, 0u, 0u, 0u);
+        int n_valid = 0;
+#pragma unroll
+        for (int j = 0; j < N; ++j) n_valid += ok[j] ? 1 : 0;
         uint32_t packed[4];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             double term[N];
-            bool val[N];
+            int emax = -1, emin = 4096;
+            bool special = false;
 #pragma unroll
             for (int j = 0; j < N; ++j) {
                 const uint32_t q = (c >> 1) == 0 ? rows[j].x
                                  : (c >> 1) == 1 ? rows[j].y
                                  : (c >> 1) == 2 ? rows[j].z : rows[j].w;
                 const float yv = (c & 1) ? bf16_hi(q) : bf16_lo(q);
-                term[j] = __dmul_rn((double)wj[j], (double)yv);  // exact
-                val[j] = ok[j];
-            }
-#pragma unroll
-            for (int pass = 0; pass < N; ++pass) {
-#pragma unroll
-                for (int i = pass & 1; i + 1 < N; i += 2) {
-                    if (canon_after(term[i], val[i], term[i + 1], val[i + 1])) {
-                        const double td = term[i];
-                        term[i] = term[i + 1];
-                        term[i + 1] = td;
-                        const bool tv = val[i];
-                        val[i] = val[i + 1];
-                        val[i + 1] = tv;
-                    }
+                term[j] = ok[j] ? __dmul_rn((double)wj[j], (double)yv) : 0.0;  // exact
+                const uint64_t b = (uint64_t)__double_as_longlong(term[j]);
+                const int e = (int)((b >> 52) & 0x7ffu);
+                if (ok[j] && e == 0x7ff) special = true;
+                if (ok[j] && (b << 1) != 0) {
+                    emax = e > emax ? e : emax;
+                    emin = e < emin ? e : emin;
                 }
             }
             double sum = 0.0;
+            if (!special && emax - emin <= 16) {
 #pragma unroll
-            for (int j = 0; j < N; ++j)
-                if (val[j]) sum = __dadd_rn(sum, term[j]);
+                for (int j = 0; j < N; ++j)
+                    if (ok[j]) sum = __dadd_rn(sum, term[j]);
+            } else {
+                uint64_t key[N];
+#pragma unroll
+                for (int j = 0; j < N; ++j) key[j] = ok[j] ? canon_key(term[j]) : ~0ull;
+#pragma unroll
+                for (int pass = 0; pass < N; ++pass) {
+#pragma unroll
+                    for (int i = pass & 1; i + 1 < N; i += 2) {
+                        const uint64_t lo = key[i] < key[i + 1] ? key[i] : key[i + 1];
+                        const uint64_t hi = key[i] < key[i + 1] ? key[i + 1] : key[i];
+                        key[i] = lo;
+                        key[i + 1] = hi;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < N; ++j)
+                    if (j < n_valid) sum = __dadd_rn(sum, from_key(key[j]));
+            }
             const float f = __double2float_rn(sum);
             if (c & 1) packed[c >> 1] |= pack_bf16(0.0f, f) & 0xffff0000u;
             else packed[c >> 1] = pack_bf16(f, 0.0f) & 0xffffu;

@@ -4,8 +4,8 @@
 // balanced), where load_e = tokens_per_expert_e / N and p_{t,e} = s_{t,e} / sum_e' s_{t,e'}
 // with s the unbiased scores of the routing contract (softmax, sigmoid or sqrtsoftplus).
 //
-// Deterministic without float atomics: block b owns 256 consecutive tokens, warp w of it
-// 32 of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
+// Deterministic without float atomics: block b owns 64 consecutive tokens, warp w of it 8
+// of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
 // ...); the 8 warp partials are added in warp order, then the block partials in block order
 // by the finishing kernel, and aux is a fixed tree over the experts. The result depends on
 // T (a batch statistic), never on scheduling.
@@ -14,7 +14,7 @@
 namespace moe {
 namespace {
 
-constexpr int kTokPerBlock = 256;
+constexpr int kTokPerBlock = 64;
 constexpr int kWarps = 8;
 constexpr int kTokPerWarp = kTokPerBlock / kWarps;
 

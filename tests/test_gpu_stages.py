@@ -269,13 +269,18 @@ def test_router_stats_against_oracle(name, T, keep):
 @pytest.mark.parametrize("T,K,H,shared,masked", [(64, 2, 128, False, True), (1000, 8, 2048, False, True),
                                                   (333, 6, 4096, True, True), (100, 16, 256, True, False),
                                                   (500, 1, 512, False, False)])
-def test_combine_invariant_bit_exact_and_order_free(T, K, H, shared, masked):
+@pytest.mark.parametrize("spread", [0.0, 2.0, 12.0])
+def test_combine_invariant_bit_exact_and_order_free(T, K, H, shared, masked, spread):
     """The order-invariant combine matches the oracle bit for bit, and permuting each
-    token's (weight, row) pairs does not change a bit (the rank-order combine does)."""
+    token's (weight, row) pairs does not change a bit (the rank-order combine does).
+    `spread`: rows scaled by 10^U(-spread, spread) -- 0 keeps nearly every element's terms
+    within 16 binary orders (the summed-as-they-come route), 12 sends most elements through
+    the sorted route."""
     rng = np.random.default_rng(T * 11 + K)
     rows = T * K
     y = (synthetic.normal_bf16(rows, H, 1.0, T + K, "x").float()
-         * torch.from_numpy(10.0 ** rng.uniform(-2, 2, (rows, 1))).float()).to(torch.bfloat16)
+         * torch.from_numpy(10.0 ** rng.uniform(-spread, spread, (rows, 1))).float()
+         ).to(torch.bfloat16)
     ys = synthetic.normal_bf16(T, H, 1.0, T + K, "fill") if shared else None
     w = rng.uniform(0, 1, (T, K)).astype(np.float32)
     dest = rng.permutation(rows).astype(np.int32).reshape(T, K)
