@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint4* __restric
                                                           uint4* __restrict__ dy,
                                                           uint4* __restrict__ dy_shared)
 {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int hv = H >> 3;  // 16-byte chunks per row
     const int warps = (gridDim.x * blockDim.x) >> 5;
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict
                                                          int renorm, float route_scale,
                                                          float* dl, uint16_t* dl_bf, int ld_bf)
 {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
@@ -199,6 +201,7 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint4* __restrict_
                                                         const uint8_t* __restrict__ mask,
                                                         int T, int K, int H, uint4* __restrict__ dx)
 {
+    pdl_wait();
     const int hv = H >> 3;
     const int64_t n = (int64_t)T * hv;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint4* __restrict_
 __global__ void __launch_bounds__(1024) padded_offsets_kernel(const int32_t* __restrict__ off,
                                                               int G, int rows, int32_t* poff)
 {
+    pdl_wait();
     __shared__ int32_t part[1024];
     const int g = threadIdx.x;
     int32_t c = 0;
@@ -261,6 +265,7 @@ __global__ void __launch_bounds__(1024) padded_offsets_kernel(const int32_t* __r
 __global__ void colmap_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
                               int G, int64_t rows_bound, int32_t* __restrict__ col)
 {
+    pdl_wait();
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows_bound;
          r += (int64_t)gridDim.x * blockDim.x) {
         if (r >= off[G]) {
@@ -286,6 +291,7 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
                                                         int64_t ld_out, int64_t out_batch,
                                                         const int32_t* __restrict__ colmap)
 {
+    pdl_wait();
     __shared__ uint16_t tile[64][65];
     const int64_t r0 = (int64_t)blockIdx.x * 64;
     const int f0 = blockIdx.y * 64;
@@ -330,6 +336,7 @@ __global__ void zero_pad_kernel(uint16_t* __restrict__ out, int F, int64_t ld_ou
                                 const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
                                 int rows)
 {
+    pdl_wait();
     const int g = blockIdx.y;
     const int64_t n = off ? (int64_t)(off[g + 1] - off[g]) : rows;
     const int64_t c0 = poff[g] + n, c1 = poff[g + 1];
@@ -351,10 +358,8 @@ cudaError_t launch_router_bwd_ne(const moe_cfg& c, const float* logits, const in
     const int cap = num_sms() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    router_bwd_kernel<NE><<<blocks, 256, 0, st>>>(logits, ids, dw, mask, c.T, c.E, c.K,
-                                                  c.score_fn, c.renorm, c.route_scale, dl,
-                                                  dl_bf, ld_bf);
-    return cudaGetLastError();
+    return launch_pdl(router_bwd_kernel<NE>, dim3(blocks), dim3(256), 0, st, logits, ids, dw, mask,
+                      c.T, c.E, c.K, c.score_fn, c.renorm, c.route_scale, dl, dl_bf, ld_bf);
 }
 
 int grid_for(int64_t work, int per_block)
@@ -371,10 +376,10 @@ cudaError_t launch_combine_bwd(const moe_cfg& c, const uint16_t* dout, const uin
                                const float* w, const int32_t* dest_row, const uint8_t* mask,
                                float* dw, uint16_t* dy, uint16_t* dy_shared, cudaStream_t st)
 {
-    combine_bwd_kernel<<<grid_for((int64_t)c.T * 32, 256), 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), w, dest_row, mask,
-        c.T, c.K, c.H, dw, reinterpret_cast<uint4*>(dy), reinterpret_cast<uint4*>(dy_shared));
-    return cudaGetLastError();
+    return launch_pdl(combine_bwd_kernel, dim3(grid_for((int64_t)c.T * 32, 256)), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), w,
+                      dest_row, mask, c.T, c.K, c.H, dw, reinterpret_cast<uint4*>(dy),
+                      reinterpret_cast<uint4*>(dy_shared));
 }
 
 cudaError_t launch_router_bwd(const moe_cfg& c, const float* logits, const int32_t* ids,
@@ -394,26 +399,26 @@ cudaError_t launch_unpermute(const moe_cfg& c, const uint16_t* rows, const int32
                              const uint16_t* shared, const uint16_t* router, const uint8_t* mask,
                              uint16_t* dx, cudaStream_t st)
 {
-    unpermute_kernel<<<grid_for((int64_t)c.T * (c.H / 8), 256), 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(rows), dest_row, reinterpret_cast<const uint4*>(shared),
-        reinterpret_cast<const uint4*>(router), mask, c.T, c.K, c.H, reinterpret_cast<uint4*>(dx));
-    return cudaGetLastError();
+    return launch_pdl(unpermute_kernel, dim3(grid_for((int64_t)c.T * (c.H / 8), 256)), dim3(256), 0,
+                      st, reinterpret_cast<const uint4*>(rows), dest_row,
+                      reinterpret_cast<const uint4*>(shared),
+                      reinterpret_cast<const uint4*>(router), mask, c.T, c.K, c.H,
+                      reinterpret_cast<uint4*>(dx));
 }
 
 cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* poff,
                                   cudaStream_t st)
 {
     if (G < 1 || G > 1024) return cudaErrorInvalidValue;
-    padded_offsets_kernel<<<1, 1024, 0, st>>>(off, G, rows, poff);
-    return cudaGetLastError();
+    return launch_pdl(padded_offsets_kernel, dim3(1), dim3(1024), 0, st, off, G, rows, poff);
 }
 
 cudaError_t launch_colmap(const int32_t* off, const int32_t* poff, int G, int64_t rows_bound,
                           int32_t* col, cudaStream_t st)
 {
     if (rows_bound <= 0) return cudaSuccess;
-    colmap_kernel<<<grid_for(rows_bound, 256), 256, 0, st>>>(off, poff, G, rows_bound, col);
-    return cudaGetLastError();
+    return launch_pdl(colmap_kernel, dim3(grid_for(rows_bound, 256)), dim3(256), 0, st, off, poff,
+                      G, rows_bound, col);
 }
 
 cudaError_t launch_transpose(const uint16_t* in, int64_t R, int F, int64_t ld_in, int64_t in_batch,
@@ -426,12 +431,10 @@ cudaError_t launch_transpose(const uint16_t* in, int64_t R, int F, int64_t ld_in
     const bool vec = (F % 8 == 0) && (ld_in % 8 == 0) &&
                      (reinterpret_cast<uintptr_t>(in) % 16 == 0) && (in_batch % 8 == 0);
     if (vec)
-        transpose_kernel<true><<<grid, 256, 0, st>>>(in, R, F, ld_in, in_batch, out, ld_out,
-                                                     out_batch, colmap);
-    else
-        transpose_kernel<false><<<grid, 256, 0, st>>>(in, R, F, ld_in, in_batch, out, ld_out,
-                                                      out_batch, colmap);
-    return cudaGetLastError();
+        return launch_pdl(transpose_kernel<true>, grid, dim3(256), 0, st, in, R, F, ld_in, in_batch,
+                          out, ld_out, out_batch, colmap);
+    return launch_pdl(transpose_kernel<false>, grid, dim3(256), 0, st, in, R, F, ld_in, in_batch,
+                      out, ld_out, out_batch, colmap);
 }
 
 cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t* off,
@@ -439,9 +442,8 @@ cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t*
 {
     if (F <= 0 || G <= 0) return cudaSuccess;
     const int bx = (int)((F * 64 + 255) / 256 < 64 ? (F * 64 + 255) / 256 : 64);
-    zero_pad_kernel<<<dim3((unsigned)bx, (unsigned)G), 256, 0, st>>>(out, F, ld_out, off, poff,
-                                                                     rows);
-    return cudaGetLastError();
+    return launch_pdl(zero_pad_kernel, dim3((unsigned)bx, (unsigned)G), dim3(256), 0, st, out, F,
+                      ld_out, off, poff, rows);
 }
 
 }  // namespace moe

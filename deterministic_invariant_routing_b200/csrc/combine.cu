@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       int K, int vec_per_row,
                                                       uint4* __restrict__ out)
 {
+    pdl_wait();
     const int64_t total = (int64_t)T * vec_per_row;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
@@ -106,10 +107,9 @@ cudaError_t launch_k(const moe_cfg& c, const uint16_t* y, const float* w, const 
     int64_t blocks = (total + 255) / 256;
     const int64_t cap = (int64_t)num_sms() * 8;
     if (blocks > cap) blocks = cap;
-    combine_kernel<KMAX><<<(unsigned)blocks, 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys), mask,
-        c.T, c.K, vec, reinterpret_cast<uint4*>(out));
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<KMAX>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys),
+                      mask, c.T, c.K, vec, reinterpret_cast<uint4*>(out));
 }
 
 // Order-invariant variant ("From Expert Reduction to Behavioral Divergence", arXiv
@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(256) combine_invariant_kernel(
     const uint4* __restrict__ y_shared, const uint8_t* __restrict__ mask, int T, int K,
     int vec_per_row, uint4* __restrict__ out)
 {
+    pdl_wait();
     constexpr int N = KMAX + 1;
     const int64_t total = (int64_t)T * vec_per_row;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
@@ -229,10 +230,9 @@ cudaError_t launch_inv(const moe_cfg& c, const uint16_t* y, const float* w, cons
     int64_t blocks = (total + 255) / 256;
     const int64_t cap = (int64_t)num_sms() * 8;
     if (blocks > cap) blocks = cap;
-    combine_invariant_kernel<KMAX><<<(unsigned)blocks, 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys), mask,
-        c.T, c.K, vec, reinterpret_cast<uint4*>(out));
-    return cudaGetLastError();
+    return launch_pdl(combine_invariant_kernel<KMAX>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys),
+                      mask, c.T, c.K, vec, reinterpret_cast<uint4*>(out));
 }
 
 }  // namespace

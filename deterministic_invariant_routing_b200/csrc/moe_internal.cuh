@@ -16,6 +16,41 @@ __device__ __forceinline__ void status_add(int32_t* status, int word, int v)
     if (status != nullptr && v != 0) atomicAdd(status + word, v);
 }
 
+// ------------------------------------------------------------------ dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: it may
+// be scheduled while the kernel before it on the stream is still finishing, so its launch
+// and setup overlap that kernel's tail. pdl_wait() blocks until the preceding grid has
+// completed and its memory is visible; every kernel calls it before its first global
+// memory access. pdl_trigger() lets the next kernel be scheduled early (a CTA that never
+// calls it triggers when it exits).
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ launchers
 
 // routing: one warp per token

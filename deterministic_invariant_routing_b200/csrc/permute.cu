@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __rest
                                                            int32_t* __restrict__ counts,
                                                            int32_t* status)
 {
+    pdl_wait();
     extern __shared__ int32_t sh[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
     __syncthreads();
@@ -63,6 +64,7 @@ __global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __rest
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, int nblocks,
                                                     int E, int32_t* __restrict__ offsets)
 {
+    pdl_wait();
     __shared__ int32_t warp_tot[32];
     const int e = threadIdx.x;
     int32_t total = 0;
@@ -110,6 +112,7 @@ __global__ void __launch_bounds__(kWarps * 32) place_kernel(const int32_t* __res
                                                             int32_t* __restrict__ dest_row,
                                                             int32_t* __restrict__ perm_token)
 {
+    pdl_wait();
     extern __shared__ int32_t wbase[];  // [kWarps][E]
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wbase[i] = 0;
@@ -158,6 +161,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
                                                      int K, int vec_per_row,
                                                      uint4* __restrict__ x_perm)
 {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t wpb = blockDim.x >> 5;
     for (int64_t t = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); t < T;
@@ -198,10 +202,12 @@ cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offset
     const int nb = (int)((A + kChunk - 1) / kChunk);
     int32_t* counts = static_cast<int32_t*>(ws);
     if (nb > 0) {
-        hist_kernel<<<nb, kWarps * 32, c.E * sizeof(int32_t), st>>>(ids, A, c.E, counts,
-                                                                    status);
+        if (const cudaError_t e = launch_pdl(hist_kernel, dim3(nb), dim3(kWarps * 32),
+                                             c.E * sizeof(int32_t), st, ids, A, c.E, counts,
+                                             status); e != cudaSuccess) return e;
     }
-    scan_kernel<<<1, 1024, 0, st>>>(counts, nb, c.E, offsets);
+    if (const cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, counts, nb, c.E,
+                                         offsets); e != cudaSuccess) return e;
     if (nb > 0) {
         const size_t smem = (size_t)kWarps * c.E * sizeof(int32_t);
         if (smem > 48 * 1024) {
@@ -210,8 +216,9 @@ cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offset
                                                  (int)smem);
             if (e != cudaSuccess) return e;
         }
-        place_kernel<<<nb, kWarps * 32, smem, st>>>(ids, A, c.K, c.E, counts, dest_row,
-                                                    perm_token);
+        if (const cudaError_t e = launch_pdl(place_kernel, dim3(nb), dim3(kWarps * 32), smem, st,
+                                             ids, A, c.K, c.E, counts, dest_row,
+                                             perm_token); e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
@@ -245,10 +252,9 @@ cudaError_t launch_gather_rows(const moe_cfg& c, const uint16_t* x, const int32_
     int64_t blocks = ((int64_t)c.T + 7) / 8;
     const int64_t cap = (int64_t)num_sms() * 16;
     if (blocks > cap) blocks = cap;
-    gather_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), dest_row,
-                                                    c.T, c.K, vec,
-                                                    reinterpret_cast<uint4*>(x_perm));
-    return cudaGetLastError();
+    return launch_pdl(gather_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(x), dest_row, c.T, c.K, vec,
+                      reinterpret_cast<uint4*>(x_perm));
 }
 
 }  // namespace moe

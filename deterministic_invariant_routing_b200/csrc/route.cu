@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     int32_t* __restrict__ ids,
                                                     float* __restrict__ w, int32_t* status)
 {
+    pdl_wait();
     extern __shared__ float choice_smem[];  // [warps][E], group-limited selection only
     const int lane = threadIdx.x & 31;
     float* cw = choice_smem + (threadIdx.x >> 5) * E;
@@ -161,10 +162,9 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bi
     if (blocks > cap) blocks = cap;
     const int n_group = c.n_group > 1 ? c.n_group : 0;
     const size_t smem = n_group ? (size_t)wpb * c.E * sizeof(float) : 0;
-    route_kernel<NE><<<blocks, threads, smem, st>>>(logits, c.T, c.E, c.K, sel_bias, mask,
-                                                    c.score_fn, c.renorm, c.route_scale, n_group,
-                                                    c.topk_group, ids, w, status);
-    return cudaGetLastError();
+    return launch_pdl(route_kernel<NE>, dim3(blocks), dim3(threads), smem, st, logits, c.T, c.E,
+                      c.K, sel_bias, mask, c.score_fn, c.renorm, c.route_scale, n_group,
+                      c.topk_group, ids, w, status);
 }
 
 }  // namespace

@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __re
                                                                float* __restrict__ partial,
                                                                int32_t* __restrict__ kept)
 {
+    pdl_wait();
     extern __shared__ float wsum[];  // [kWarps][E]
     __shared__ int32_t wkept[kWarps];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(1024) stats_finish_kernel(const float* __restr
                                                             float* __restrict__ mean_prob,
                                                             float* __restrict__ aux)
 {
+    pdl_wait();
     __shared__ float wsum[32];
     const int e = threadIdx.x, lane = e & 31, wid = e >> 5;
     int64_t n = 0;
@@ -119,9 +121,8 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const uint8_t* mask
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
-    prob_sum_kernel<NE><<<nb, kWarps * 32, smem, st>>>(logits, mask, c.T, c.E, c.score_fn,
-                                                       partial, kept);
-    return cudaGetLastError();
+    return launch_pdl(prob_sum_kernel<NE>, dim3(nb), dim3(kWarps * 32), smem, st, logits, mask, c.T,
+                      c.E, c.score_fn, partial, kept);
 }
 
 }  // namespace
@@ -152,9 +153,8 @@ cudaError_t launch_router_stats(const moe_cfg& c, const float* logits, const uin
         else err = launch_ne<32>(c, logits, mask, partial, kept, nb, st);
         if (err != cudaSuccess) return err;
     }
-    stats_finish_kernel<<<1, 1024, 0, st>>>(partial, kept, nb, c.E, offsets, counts, mean_prob,
-                                            aux);
-    return cudaGetLastError();
+    return launch_pdl(stats_finish_kernel, dim3(1), dim3(1024), 0, st, partial, kept, nb, c.E,
+                      offsets, counts, mean_prob, aux);
 }
 
 }  // namespace moe

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
+    pdl_wait();  // the previous kernel's writes are visible from here on
 
     if (warp == 0) {
         if (lane == 0) {
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
             }
+            pdl_trigger();  // every load is issued: the next kernel may be scheduled
             if (*abort_flag) {
                 // let every copy this thread started land before the CTA exits
                 for (int s = 0; s < S; ++s)
@@ -253,8 +255,7 @@ cudaError_t launch_router_variant(const RouterProblem& p, cudaStream_t st)
     int grid = num_sms();
     if (tiles < grid) grid = (int)tiles;
     if (grid < 1) grid = 1;
-    kernel<<<grid, kThreads, C::kSmem, st>>>(ma, mb, a);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, st, ma, mb, a);
 }
 
 }  // namespace

@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
+    pdl_wait();  // the previous kernel's writes (offsets, operands) are visible from here on
     if (warp == 2) {
         auto row_off = [&](int g) -> int {
             return args.offsets ? args.offsets[g] : (g == 0 ? 0 : args.rows);
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 }
                 if (!ok) break;
             }
+            pdl_trigger();  // every load is issued: the next kernel may be scheduled
             if (*abort_flag && leader) {
                 for (int s = 0; s < S; ++s)
                     if (armed & (1u << s))
@@ -573,16 +575,18 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     static int max_clusters[64] = {};
     static size_t max_smem[64] = {};
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kThreads2, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
@@ -592,8 +596,10 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (max_clusters[dev] == 0 || smem > max_smem[dev]) {
         // co-resident clusters at this shared-memory size (one CTA per SM in practice)
         cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.numAttrs = 1;  // the cluster shape only
         int n = 0;
         err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+        cfg.numAttrs = 2;
         if (err != cudaSuccess) return err;
         if (n <= 0) return cudaErrorInvalidConfiguration;
         max_clusters[dev] = n;
