@@ -105,7 +105,7 @@ cudaError_t launch_k(const moe_cfg& c, const uint16_t* y, const float* w, const 
     const int vec = c.H / 8;
     const int64_t total = (int64_t)c.T * vec;
     int64_t blocks = (total + 255) / 256;
-    const int64_t cap = (int64_t)num_sms() * 8;
+    const int64_t cap = resident_blocks((const void*)combine_kernel<KMAX>, 256, 0);
     if (blocks > cap) blocks = cap;
     return launch_pdl(combine_kernel<KMAX>, dim3((unsigned)blocks), dim3(256), 0, st,
                       reinterpret_cast<const uint4*>(y), w, dr, reinterpret_cast<const uint4*>(ys),

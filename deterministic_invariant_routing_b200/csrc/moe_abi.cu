@@ -23,6 +23,16 @@ int num_sms()
     return n;
 }
 
+int resident_blocks(const void* kernel, int threads, size_t smem)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    return num_sms() * per_sm;
+}
+
 bool device_is_sm100()
 {
     int dev = 0, major = 0, minor = 0;

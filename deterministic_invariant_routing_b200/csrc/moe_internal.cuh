@@ -154,5 +154,8 @@ cudaError_t launch_router(const RouterProblem& p, cudaStream_t st);
 // device facts
 int num_sms();
 bool device_is_sm100();
+// blocks of `kernel` resident on the whole GPU at once (grid-stride kernels launched with
+// exactly this many run as one wave)
+int resident_blocks(const void* kernel, int threads, size_t smem);
 
 }  // namespace moe
