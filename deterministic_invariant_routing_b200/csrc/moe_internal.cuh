@@ -113,7 +113,14 @@ cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t*
 //                   out[r, c] = bf16(dh * u * silu'(g)), out[r, n + c] = bf16(dh * silu(g))
 //   EPI_WGRAD       grouped over K: out[g][m, c] = fp32(sum over k in [k_offsets[g],
 //                   k_offsets[g+1]) of A[m, k] * B[c, k]) -- an expert's rows contracted
-enum GemmEpilogue { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
+//   EPI_F32         out[r, c] = fp32(A . B^T) + bias[c] (one rounded add; bias NULL: + 0)
+enum GemmEpilogue {
+    EPI_SWIGLU = 0,
+    EPI_BF16 = 1,
+    EPI_SWIGLU_BWD = 2,
+    EPI_WGRAD = 3,
+    EPI_F32 = 4
+};
 
 struct GemmProblem {
     int epilogue;            // GemmEpilogue
@@ -130,7 +137,7 @@ struct GemmProblem {
     int rows;                // rows when offsets == NULL (EPI_WGRAD: rows of A = M)
     void* out;               // output [*, ldo]
     int64_t ldo;             // output row stride in elements
-    const float* bias;       // unused by the pair kernel
+    const float* bias;       // EPI_F32: per-column bias or NULL
     int32_t* status;         // device status words (MOE_ST_PIPE_TIMEOUT) or NULL
     const uint16_t* aux;     // EPI_SWIGLU_BWD: dh [rows, ld_aux] bf16
     int64_t ld_aux;

@@ -263,6 +263,26 @@ cudaError_t launch_router_variant(const RouterProblem& p, cudaStream_t st)
 cudaError_t launch_router(const RouterProblem& p, cudaStream_t st)
 {
     if (p.H % BK != 0 || p.logits == nullptr) return cudaErrorInvalidValue;
+    if (p.E % 128 == 0) {
+        // whole 128-expert column tiles: the CTA-pair kernel, each SM loading half of the
+        // router rows per k-block (the rows every tile shares)
+        GemmProblem g{};
+        g.epilogue = EPI_F32;
+        g.a = p.x;
+        g.a_rows = p.T;
+        g.a_rows_total = p.T;
+        g.b = p.w_router;
+        g.b_rows_per_group = p.E;
+        g.k = p.H;
+        g.n = p.E;
+        g.groups = 1;
+        g.rows = p.T;
+        g.out = p.logits;
+        g.ldo = p.E;
+        g.bias = p.logit_bias;
+        g.status = p.status;
+        return launch_tc_gemm_pair(g, st);
+    }
     // N = next power of two >= E, at least 32, at most 256 (column tiles beyond)
     if (p.E <= 32) return launch_router_variant<32>(p, st);
     if (p.E <= 64) return launch_router_variant<64>(p, st);

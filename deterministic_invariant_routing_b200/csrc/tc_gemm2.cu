@@ -64,6 +64,7 @@ struct PairArgs {
     const uint16_t* aux;         // EPI_SWIGLU_BWD: dh
     int64_t ld_aux;
     int half_out;                // EPI_SWIGLU_BWD: column of the first up gradient
+    const float* bias;           // EPI_F32: per-column bias or NULL
 };
 
 template <int EPI, int NP>
@@ -513,6 +514,26 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     const int ucol = args.half_out + col;
                     store_block(pu, full_blk, valid, row_blk, ucol, out + grow * args.ldo + ucol);
                 }
+            } else if (EPI == EPI_F32) {
+                // fp32 rows plus the column bias (the router's logits)
+                float* o = static_cast<float*>(args.out);
+#pragma unroll 1
+                for (int c = 0; c < NP; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + (uint32_t)c, r);
+                    const int col = ti.n * NP + c;
+                    if (valid) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = __fadd_rn(__uint_as_float(r[j]),
+                                             args.bias != nullptr ? args.bias[col + j] : 0.0f);
+                        float4* dst = reinterpret_cast<float4*>(o + grow * args.ldo + col);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                }
             } else if (EPI == EPI_WGRAD) {
                 // fp32 weight gradient rows of group g; a group with no rows gives zeros
                 float* o = static_cast<float*>(args.out);
@@ -612,7 +633,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (!make_map(&mb, p.b, wgrad ? (int64_t)p.n : (int64_t)groups * p.b_rows_per_group, p.k,
                   NP / 2))
         return cudaErrorInvalidValue;
-    if (wgrad) {
+    if (wgrad || EPI == EPI_F32) {
         mo = mb;  // fp32 rows are stored from registers; the store map is not used
     } else {
         const int out_cols = (EPI == EPI_SWIGLU_BWD) ? 2 * p.n : p.n;
@@ -633,6 +654,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.aux = p.aux;
     a.ld_aux = p.ld_aux;
     a.half_out = (EPI == EPI_SWIGLU_BWD) ? p.n : 0;
+    a.bias = p.bias;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;
@@ -667,6 +689,11 @@ cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st)
         if (p.k_offsets == nullptr || p.rows < 1) return cudaErrorInvalidValue;
         if (p.n % 256 == 0) return launch_pair_variant<EPI_WGRAD, 256, false>(p, st);
         if (p.n % 128 == 0) return launch_pair_variant<EPI_WGRAD, 128, false>(p, st);
+        return cudaErrorInvalidValue;
+    }
+    if (p.epilogue == EPI_F32) {
+        if (p.n % 256 == 0) return launch_pair_variant<EPI_F32, 256, false>(p, st);
+        if (p.n % 128 == 0) return launch_pair_variant<EPI_F32, 128, false>(p, st);
         return cudaErrorInvalidValue;
     }
     if (p.epilogue == EPI_BF16) {
