@@ -21,11 +21,6 @@
 namespace moe {
 namespace {
 
-__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b)
-{
-    return a > b ? a : b;
-}
-
 __device__ __forceinline__ unsigned long long select_key(float c, int id)
 {
     return ((unsigned long long)order_bits(c) << 32) |
@@ -113,24 +108,38 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                 if (e < E && ((kept >> (e / gs)) & 1u) == 0u) key[i] = 0ull;
             }
         }
-        // K rounds of a warp-wide arg-max over the remaining keys
+        // each lane orders its own keys (descending, scores alongside) once; then K rounds
+        // of a warp arg-max over the lanes' heads, the winning lane dropping its head
+        float sv[NE];
+#pragma unroll
+        for (int i = 0; i < NE; ++i) sv[i] = s[i];
+#pragma unroll
+        for (int pass = 0; pass < NE; ++pass) {
+#pragma unroll
+            for (int i = pass & 1; i + 1 < NE; i += 2) {
+                const bool swap = key[i] < key[i + 1];
+                const unsigned long long k0 = key[i], k1 = key[i + 1];
+                const float s0 = sv[i], s1 = sv[i + 1];
+                key[i] = swap ? k1 : k0;
+                key[i + 1] = swap ? k0 : k1;
+                sv[i] = swap ? s1 : s0;
+                sv[i + 1] = swap ? s0 : s1;
+            }
+        }
         int my_id = -1;
         float my_s = 0.0f, den = 0.0f;
         for (int j = 0; j < K; ++j) {
-            unsigned long long best = 0ull;
+            const int e = warp_argmax_id(key[0]);
+            const int owner = e & 31;
+            const float se = __shfl_sync(0xffffffffu, sv[0], owner);
+            if (lane == owner) {
 #pragma unroll
-            for (int i = 0; i < NE; ++i) best = umax64(best, key[i]);
-            const int e = warp_argmax_id(best);
-            const int owner = e & 31, slot = e >> 5;
-            float se = 0.0f;
-#pragma unroll
-            for (int i = 0; i < NE; ++i) {
-                if (lane == owner && i == slot) {
-                    se = s[i];
-                    key[i] = 0ull;
+                for (int i = 0; i + 1 < NE; ++i) {
+                    key[i] = key[i + 1];
+                    sv[i] = sv[i + 1];
                 }
+                key[NE - 1] = 0ull;
             }
-            se = __shfl_sync(0xffffffffu, se, owner);
             den = (j == 0) ? se : __fadd_rn(den, se);
             if (lane == j) { my_id = e; my_s = se; }
         }
