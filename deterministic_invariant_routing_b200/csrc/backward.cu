@@ -11,9 +11,9 @@
 //                     fixed fp32 order (see router_bwd_kernel)
 //  un-permute         dx_t = bf16(rank-order sum of the token's row gradients, then the
 //                     shared expert's and the router's terms); masked tokens +0
-//  transposes         [R, F] -> [F, columns] bf16, rows optionally mapped to padded per-expert
-//                     column ranges (the K operand layout of the weight-gradient products),
-//                     padding columns zeroed
+//  padded layout      each expert's dispatch rows start at a multiple of 64 (padding rows
+//                     zero), so its rows are whole 64-row K blocks of the weight-gradient
+//                     products, which read the row-major activations in place (MN-major)
 //
 // Nothing here uses float atomics; every reduction has a fixed order, so results are
 // bitwise repeatable and a token's input gradient does not depend on the other tokens.
@@ -261,92 +261,31 @@ __global__ void __launch_bounds__(1024) padded_offsets_kernel(const int32_t* __r
     if (g == 0) poff[0] = 0;
 }
 
-// column of each grouped row in the padded layout (-1 past the last routed row)
-__global__ void colmap_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
-                              int G, int64_t rows_bound, int32_t* __restrict__ col)
-{
-    pdl_wait();
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows_bound;
-         r += (int64_t)gridDim.x * blockDim.x) {
-        if (r >= off[G]) {
-            col[r] = -1;
-            continue;
-        }
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (off[mid] <= r) lo = mid;
-            else hi = mid - 1;
-        }
-        col[r] = (int32_t)(poff[lo] + (r - off[lo]));
-    }
-}
-
-// out[z][f, col(r)] = in[z][r, f] for a 64 x 64 tile per block; col(r) = colmap[r] (skip
-// when < 0) or r. VEC: F and ld_in are multiples of 8 (16-byte loads).
-template <bool VEC>
-__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ in,
-                                                        int64_t R, int F, int64_t ld_in,
-                                                        int64_t in_batch, uint16_t* __restrict__ out,
-                                                        int64_t ld_out, int64_t out_batch,
-                                                        const int32_t* __restrict__ colmap)
-{
-    pdl_wait();
-    __shared__ uint16_t tile[64][65];
-    const int64_t r0 = (int64_t)blockIdx.x * 64;
-    const int f0 = blockIdx.y * 64;
-    const uint16_t* src = in + (int64_t)blockIdx.z * in_batch;
-    uint16_t* dst = out + (int64_t)blockIdx.z * out_batch;
-    if (VEC) {
-        for (int idx = threadIdx.x; idx < 64 * 8; idx += 256) {
-            const int rr = idx >> 3, vv = idx & 7;
-            const int64_t r = r0 + rr;
-            const int f = f0 + vv * 8;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < R && f < F) v = *reinterpret_cast<const uint4*>(src + r * ld_in + f);
-            const uint32_t q[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                tile[rr][vv * 8 + 2 * e] = (uint16_t)(q[e] & 0xffffu);
-                tile[rr][vv * 8 + 2 * e + 1] = (uint16_t)(q[e] >> 16);
-            }
-        }
-    } else {
-        for (int idx = threadIdx.x; idx < 64 * 64; idx += 256) {
-            const int rr = idx >> 6, ff = idx & 63;
-            const int64_t r = r0 + rr;
-            const int f = f0 + ff;
-            tile[rr][ff] = (r < R && f < F) ? src[r * ld_in + f] : (uint16_t)0;
-        }
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < 64 * 64; idx += 256) {
-        const int ff = idx >> 6, rr = idx & 63;
-        const int64_t r = r0 + rr;
-        const int f = f0 + ff;
-        if (r >= R || f >= F) continue;
-        const int64_t c = colmap ? (int64_t)colmap[r] : r;
-        if (c >= 0) dst[(int64_t)f * ld_out + c] = tile[rr][ff];
-    }
-}
-
-// zero the padding columns [poff[g] + n_g, poff[g+1]) of every row f < F of out [F, ld_out];
-// n_g = off[g+1] - off[g] (off == NULL: one group of `rows` rows)
-__global__ void zero_pad_kernel(uint16_t* __restrict__ out, int F, int64_t ld_out,
+__global__ void pad_rows_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ dest,
                                 const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
-                                int rows)
+                                int64_t A, int E, int32_t* __restrict__ dest_pad)
+{
+    pdl_wait();
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A;
+         a += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = dest[a];
+        const int32_t e = ids[a];
+        dest_pad[a] = (r >= 0 && e >= 0 && e < E) ? poff[e] + (r - off[e]) : -1;
+    }
+}
+
+// block (x, g): 16-byte chunks of group g's padding rows
+__global__ void zero_pad_rows_kernel(uint4* __restrict__ buf, int64_t vec_per_row,
+                                     const int32_t* __restrict__ off,
+                                     const int32_t* __restrict__ poff)
 {
     pdl_wait();
     const int g = blockIdx.y;
-    const int64_t n = off ? (int64_t)(off[g + 1] - off[g]) : rows;
-    const int64_t c0 = poff[g] + n, c1 = poff[g + 1];
-    const int width = (int)(c1 - c0);  // < 64
-    if (width <= 0) return;
-    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < F * 64;
-         idx += gridDim.x * blockDim.x) {
-        const int f = idx >> 6, c = idx & 63;
-        if (c < width) out[(int64_t)f * ld_out + c0 + c] = 0;
-    }
+    const int64_t r0 = (int64_t)poff[g] + (off[g + 1] - off[g]);
+    const int64_t n = ((int64_t)poff[g + 1] - r0) * vec_per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        buf[r0 * vec_per_row + i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 template <int NE>
@@ -413,37 +352,25 @@ cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* 
     return launch_pdl(padded_offsets_kernel, dim3(1), dim3(1024), 0, st, off, G, rows, poff);
 }
 
-cudaError_t launch_colmap(const int32_t* off, const int32_t* poff, int G, int64_t rows_bound,
-                          int32_t* col, cudaStream_t st)
+cudaError_t launch_pad_rows(const int32_t* ids, const int32_t* dest_row, const int32_t* off,
+                            const int32_t* poff, int64_t A, int E, int32_t* dest_pad,
+                            cudaStream_t st)
 {
-    if (rows_bound <= 0) return cudaSuccess;
-    return launch_pdl(colmap_kernel, dim3(grid_for(rows_bound, 256)), dim3(256), 0, st, off, poff,
-                      G, rows_bound, col);
+    if (A <= 0) return cudaSuccess;
+    return launch_pdl(pad_rows_kernel, dim3(grid_for(A, 256)), dim3(256), 0, st, ids, dest_row,
+                      off, poff, A, E, dest_pad);
 }
 
-cudaError_t launch_transpose(const uint16_t* in, int64_t R, int F, int64_t ld_in, int64_t in_batch,
-                             uint16_t* out, int64_t ld_out, int64_t out_batch, int batches,
-                             const int32_t* colmap, cudaStream_t st)
+cudaError_t launch_zero_pad_rows(uint16_t* buf, int64_t cols, const int32_t* off,
+                                 const int32_t* poff, int G, cudaStream_t st)
 {
-    if (R <= 0 || F <= 0 || batches <= 0) return cudaSuccess;
-    const dim3 grid((unsigned)((R + 63) / 64), (unsigned)((F + 63) / 64), (unsigned)batches);
-    if (grid.x > 2147483647u || grid.y > 65535u || grid.z > 65535u) return cudaErrorInvalidValue;
-    const bool vec = (F % 8 == 0) && (ld_in % 8 == 0) &&
-                     (reinterpret_cast<uintptr_t>(in) % 16 == 0) && (in_batch % 8 == 0);
-    if (vec)
-        return launch_pdl(transpose_kernel<true>, grid, dim3(256), 0, st, in, R, F, ld_in, in_batch,
-                          out, ld_out, out_batch, colmap);
-    return launch_pdl(transpose_kernel<false>, grid, dim3(256), 0, st, in, R, F, ld_in, in_batch,
-                      out, ld_out, out_batch, colmap);
-}
-
-cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t* off,
-                            const int32_t* poff, int G, int rows, cudaStream_t st)
-{
-    if (F <= 0 || G <= 0) return cudaSuccess;
-    const int bx = (int)((F * 64 + 255) / 256 < 64 ? (F * 64 + 255) / 256 : 64);
-    return launch_pdl(zero_pad_kernel, dim3((unsigned)bx, (unsigned)G), dim3(256), 0, st, out, F,
-                      ld_out, off, poff, rows);
+    if (G <= 0 || cols % 8 != 0) return cols % 8 ? cudaErrorInvalidValue : cudaSuccess;
+    const int64_t vec = cols / 8;
+    int bx = (int)((63 * vec + 255) / 256);
+    if (bx > 64) bx = 64;
+    if (bx < 1) bx = 1;
+    return launch_pdl(zero_pad_rows_kernel, dim3((unsigned)bx, (unsigned)G), dim3(256), 0, st,
+                      reinterpret_cast<uint4*>(buf), vec, off, poff);
 }
 
 }  // namespace moe

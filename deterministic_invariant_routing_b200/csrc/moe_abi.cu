@@ -208,10 +208,11 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     return launch_tc_gemm_pair(p, st);
 }
 
-// a grouped bf16 product: out[r] = a_r . B_g^T, B_g = b[g] of [n, k]
-cudaError_t gemm_bf16(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
-                      int rows, const uint16_t* b, int n, int k, uint16_t* out, int32_t* status,
-                      cudaStream_t st)
+// a grouped bf16 product out[r] = a_r . b[g] with b[g] = [b_k_rows, n] (N contiguous): the
+// weight as stored, read MN-major by the tensor cores (no transposed copy)
+cudaError_t gemm_bf16_mn(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                         int rows, const uint16_t* b, int n, int k, int b_k_rows, uint16_t* out,
+                         int32_t* status, cudaStream_t st)
 {
     GemmProblem p{};
     p.epilogue = EPI_BF16;
@@ -220,6 +221,8 @@ cudaError_t gemm_bf16(const uint16_t* a, int64_t a_rows, const int32_t* offsets,
     p.a_rows_total = a_rows;
     p.b = b;
     p.b_rows_per_group = n;
+    p.b_mn = 1;
+    p.b_k_rows = b_k_rows;
     p.k = k;
     p.n = n;
     p.groups = groups;
@@ -253,28 +256,6 @@ cudaError_t gemm_swiglu_bwd(const uint16_t* a, int64_t a_rows, const int32_t* of
     p.ldo = 2 * I;
     p.aux = dh;
     p.ld_aux = I;
-    p.status = status;
-    return launch_tc_gemm_pair(p, st);
-}
-
-// weight gradient of each group: out[g] [m, n] = sum over the group's K columns of
-// a[m, k] b[n, k] (fp32); a [m, kcols], b [n, kcols], K ranges k_offsets (multiples of 64)
-cudaError_t gemm_wgrad(const uint16_t* a, int m, const uint16_t* b, int n, int64_t kcols,
-                       const int32_t* k_offsets, int groups, float* out, int32_t* status,
-                       cudaStream_t st)
-{
-    GemmProblem p{};
-    p.epilogue = EPI_WGRAD;
-    p.a = a;
-    p.a_rows = m;
-    p.b = b;
-    p.k = (int)kcols;
-    p.n = n;
-    p.groups = groups;
-    p.rows = m;
-    p.out = out;
-    p.ldo = n;
-    p.k_offsets = k_offsets;
     p.status = status;
     return launch_tc_gemm_pair(p, st);
 }
@@ -420,12 +401,13 @@ cudaError_t host_pipe(HostPipe** out)
 
 size_t pad64(size_t v) { return (v + 63) / 64 * 64; }
 
-// scratch of moe_backward
+// scratch of moe_backward. The routed rows live in a padded layout: expert e's rows start at
+// poff[e] (its count rounded up to 64, the padding rows zero), so that every expert's rows
+// form whole 64-row K blocks of the weight-gradient products.
 struct BwdLayout {
-    size_t offsets, perm_token, dest_row, perm_ws, x_perm, h, y, dy, dh, dgu, dx_perm, w2t, w13t,
-        wrt, poffE, dw_tk, dl, dl_bf, dx_r, poff, colmap, dyT, hT, dguT, xpT, poffT, dlT, xT,
-        h_s, dh_s, dgu_s, dx_s, dy_s, w2st, w13st, dysT, hsT, dgusT, total;
-    int64_t rp, tp, e_pad;
+    size_t offsets, perm_token, dest_row, dest_pad, poff, perm_ws, x_perm, h, y, dy, dh, dgu,
+        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, dh_s, dgu_s, dx_s, dy_s, total;
+    int64_t rp, e_pad;
 };
 
 BwdLayout bwd_layout(const moe_cfg& c)
@@ -433,9 +415,8 @@ BwdLayout bwd_layout(const moe_cfg& c)
     BwdLayout L{};
     const size_t A = (size_t)c.T * c.K, H = c.H, I = c.I, Is = c.I_shared, T = c.T;
     L.e_pad = (int64_t)pad64(c.E);
-    L.tp = (int64_t)pad64(T > 0 ? T : 1);
     L.rp = (int64_t)pad64(A + (size_t)63 * c.E);
-    const size_t rp = (size_t)L.rp, tp = (size_t)L.tp, ep = (size_t)L.e_pad;
+    const size_t rp = (size_t)L.rp, ep = (size_t)L.e_pad;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
@@ -445,43 +426,52 @@ BwdLayout bwd_layout(const moe_cfg& c)
     L.offsets = take((c.E + 1) * 4);
     L.perm_token = take(A * 4);
     L.dest_row = take(A * 4);
+    L.dest_pad = take(A * 4);
+    L.poff = take((c.E + 1) * 4);
     L.perm_ws = take(permute_ws_bytes(c));
-    L.x_perm = take(A * H * 2);
-    L.h = take(A * I * 2);
-    L.y = take(A * H * 2);
-    L.dy = take(A * H * 2);
-    L.dh = take(A * I * 2);
-    L.dgu = take(A * 2 * I * 2);
-    L.dx_perm = take(A * H * 2);
-    L.w2t = take((size_t)c.E * I * H * 2);
-    L.w13t = take((size_t)c.E * H * 2 * I * 2);
-    L.wrt = take(H * ep * 2);
-    L.poffE = take(2 * 4);
+    L.x_perm = take(rp * H * 2);
+    L.h = take(rp * I * 2);
+    L.y = take(rp * H * 2);
+    L.dy = take(rp * H * 2);
+    L.dh = take(rp * I * 2);
+    L.dgu = take(rp * 2 * I * 2);
+    L.dx_perm = take(rp * H * 2);
     L.dw_tk = take(A * 4);
     L.dl = take(T * c.E * 4);
     L.dl_bf = take(T * ep * 2);
     L.dx_r = take(T * H * 2);
-    L.poff = take((c.E + 1) * 4);
-    L.colmap = take(A * 4);
-    L.dyT = take(H * rp * 2);
-    L.hT = take(I * rp * 2);
-    L.dguT = take(2 * I * rp * 2);
-    L.xpT = take(H * rp * 2);
-    L.poffT = take(2 * 4);
-    L.dlT = take(ep * tp * 2);
-    L.xT = take(H * tp * 2);
+    L.koffT = take(2 * 4);
     L.h_s = take(T * Is * 2);
     L.dh_s = take(T * Is * 2);
     L.dgu_s = take(T * 2 * Is * 2);
     L.dx_s = take(Is ? T * H * 2 : 0);
     L.dy_s = take(Is ? T * H * 2 : 0);
-    L.w2st = take(Is * H * 2);
-    L.w13st = take(H * 2 * Is * 2);
-    L.dysT = take(Is ? H * tp * 2 : 0);
-    L.hsT = take(Is * tp * 2);
-    L.dgusT = take(2 * Is * tp * 2);
     L.total = off;
     return L;
+}
+
+// weight gradient with both operands read MN-major in place: out[g] [m, n] = sum over the
+// group's K rows of a[k, m] b[k, n]; a [k_rows, a_cols], b [k_rows, n]
+cudaError_t gemm_wgrad_mn(const uint16_t* a, int64_t a_cols, int m, const uint16_t* b, int n,
+                          int64_t k_rows, const int32_t* k_offsets, int groups, float* out,
+                          int32_t* status, cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_WGRAD;
+    p.a = a;
+    p.a_rows = a_cols;
+    p.a_mn = 1;
+    p.b = b;
+    p.b_mn = 1;
+    p.k = (int)k_rows;
+    p.n = n;
+    p.groups = groups;
+    p.rows = m;
+    p.out = out;
+    p.ldo = n;
+    p.k_offsets = k_offsets;
+    p.status = status;
+    return launch_tc_gemm_pair(p, st);
 }
 
 #define MOE_TRY(call)                                   \
@@ -501,9 +491,12 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     const int64_t A = (int64_t)c.T * c.K;
     const int H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
     const int ep = (int)L.e_pad;
+    const int64_t rp = L.rp;
     const bool shared = Is > 0;
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* dest_row = at<int32_t>(ws, L.dest_row);
+    int32_t* dest_pad = at<int32_t>(ws, L.dest_pad);
+    int32_t* poff = at<int32_t>(ws, L.poff);
     uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
     uint16_t* h = at<uint16_t>(ws, L.h);
     uint16_t* y = at<uint16_t>(ws, L.y);
@@ -511,51 +504,39 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     uint16_t* dh = at<uint16_t>(ws, L.dh);
     uint16_t* dgu = at<uint16_t>(ws, L.dgu);
     uint16_t* dx_perm = at<uint16_t>(ws, L.dx_perm);
-    uint16_t* w2t = at<uint16_t>(ws, L.w2t);
-    uint16_t* w13t = at<uint16_t>(ws, L.w13t);
-    uint16_t* wrt = at<uint16_t>(ws, L.wrt);
-    int32_t* poffE = at<int32_t>(ws, L.poffE);
     float* dw_tk = d_topk_w ? d_topk_w : at<float>(ws, L.dw_tk);
     float* dl = dlogits ? dlogits : at<float>(ws, L.dl);
     uint16_t* dl_bf = at<uint16_t>(ws, L.dl_bf);
     uint16_t* dx_r = at<uint16_t>(ws, L.dx_r);
-    int32_t* poff = at<int32_t>(ws, L.poff);
-    int32_t* colmap = at<int32_t>(ws, L.colmap);
-    uint16_t* dyT = at<uint16_t>(ws, L.dyT);
-    uint16_t* hT = at<uint16_t>(ws, L.hT);
-    uint16_t* dguT = at<uint16_t>(ws, L.dguT);
-    uint16_t* xpT = at<uint16_t>(ws, L.xpT);
-    int32_t* poffT = at<int32_t>(ws, L.poffT);
-    uint16_t* dlT = at<uint16_t>(ws, L.dlT);
-    uint16_t* xT = at<uint16_t>(ws, L.xT);
-    const int64_t rp = L.rp, tp = L.tp;
+    int32_t* koffT = at<int32_t>(ws, L.koffT);
 
-    // dispatch and the forward intermediates, recomputed (same kernels, same bits)
+    // dispatch, then the padded row layout (expert ranges at poff, padding rows zero)
     MOE_TRY(launch_permute(c, ids, offsets, at<int32_t>(ws, L.perm_token), dest_row, status,
                            at<void>(ws, L.perm_ws), st));
-    MOE_TRY(launch_gather_rows(c, x, dest_row, x_perm, st));
-    MOE_TRY(gate_up(x_perm, A, nullptr, A, offsets, E, 0, w13, H, I, h, status, st));
-    MOE_TRY(down(h, A, offsets, E, 0, w2, H, I, y, status, st));
+    MOE_TRY(launch_padded_offsets(offsets, E, 0, poff, st));
+    MOE_TRY(launch_pad_rows(ids, dest_row, offsets, poff, A, E, dest_pad, st));
+    MOE_TRY(launch_zero_pad_rows(x_perm, H, offsets, poff, E, st));
+    MOE_TRY(launch_zero_pad_rows(dy, H, offsets, poff, E, st));
+    MOE_TRY(launch_gather_rows(c, x, dest_pad, x_perm, st));
+    // the forward intermediates recomputed (the same products: a row's bits do not depend on
+    // where it sits); padding rows give h = 0, y = 0
+    MOE_TRY(gate_up(x_perm, rp, nullptr, rp, poff, E, 0, w13, H, I, h, status, st));
+    MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, y, status, st));
 
     // combine backward: routing-weight gradients and the expert-output gradients
     uint16_t* dy_s = shared ? at<uint16_t>(ws, L.dy_s) : nullptr;
-    MOE_TRY(launch_combine_bwd(c, dout, y, topk_w, dest_row, mask, dw_tk, dy, dy_s, st));
+    MOE_TRY(launch_combine_bwd(c, dout, y, topk_w, dest_pad, mask, dw_tk, dy, dy_s, st));
 
     // routed experts: dh = dy . W2, dgu (SwiGLU backward on the recomputed gate/up
-    // product), dx rows = dgu . W13; the weights as K-major operands ([I,H] and [H,2I])
-    MOE_TRY(launch_transpose(w2, H, I, I, (int64_t)H * I, w2t, H, (int64_t)I * H, E, nullptr, st));
-    MOE_TRY(launch_transpose(w13, 2 * I, H, H, (int64_t)2 * I * H, w13t, 2 * I,
-                             (int64_t)H * 2 * I, E, nullptr, st));
-    MOE_TRY(gemm_bf16(dy, A, offsets, E, 0, w2t, I, H, dh, status, st));
-    MOE_TRY(gemm_swiglu_bwd(x_perm, A, offsets, E, 0, w13, H, I, dh, dgu, status, st));
-    MOE_TRY(gemm_bf16(dgu, A, offsets, E, 0, w13t, H, 2 * I, dx_perm, status, st));
+    // product), dx rows = dgu . W13; the weights are read MN-major as stored
+    MOE_TRY(gemm_bf16_mn(dy, rp, poff, E, 0, w2, I, H, H, dh, status, st));
+    MOE_TRY(gemm_swiglu_bwd(x_perm, rp, poff, E, 0, w13, H, I, dh, dgu, status, st));
+    MOE_TRY(gemm_bf16_mn(dgu, rp, poff, E, 0, w13, H, 2 * I, 2 * I, dx_perm, status, st));
 
-    // router: dlogits, then dx_router = bf16(dlogits) . W_router
+    // router: dlogits, then dx_router = bf16(dlogits) . W_router (K padded to 64: the rows
+    // of W_router past E read as zeros)
     MOE_TRY(launch_router_bwd(c, logits, ids, dw_tk, mask, dl, dl_bf, ep, st));
-    MOE_TRY(launch_padded_offsets(nullptr, 1, E, poffE, st));
-    MOE_TRY(launch_transpose(wr, E, H, H, 0, wrt, ep, 0, 1, nullptr, st));
-    MOE_TRY(launch_zero_pad(wrt, H, ep, nullptr, poffE, 1, E, st));
-    MOE_TRY(gemm_bf16(dl_bf, T, nullptr, 1, T, wrt, H, ep, dx_r, status, st));
+    MOE_TRY(gemm_bf16_mn(dl_bf, T, nullptr, 1, T, wr, H, ep, E, dx_r, status, st));
 
     // shared expert (all kept tokens, dy_shared = dout)
     uint16_t *h_s = nullptr, *dgu_s = nullptr, *dx_s = nullptr;
@@ -564,53 +545,25 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
         uint16_t* dh_s = at<uint16_t>(ws, L.dh_s);
         dgu_s = at<uint16_t>(ws, L.dgu_s);
         dx_s = at<uint16_t>(ws, L.dx_s);
-        uint16_t* w2st = at<uint16_t>(ws, L.w2st);
-        uint16_t* w13st = at<uint16_t>(ws, L.w13st);
         MOE_TRY(gate_up(x, T, nullptr, T, nullptr, 1, T, w13s, H, Is, h_s, status, st));
-        MOE_TRY(launch_transpose(w2s, H, Is, Is, 0, w2st, H, 0, 1, nullptr, st));
-        MOE_TRY(launch_transpose(w13s, 2 * Is, H, H, 0, w13st, 2 * Is, 0, 1, nullptr, st));
-        MOE_TRY(gemm_bf16(dy_s, T, nullptr, 1, T, w2st, Is, H, dh_s, status, st));
+        MOE_TRY(gemm_bf16_mn(dy_s, T, nullptr, 1, T, w2s, Is, H, H, dh_s, status, st));
         MOE_TRY(gemm_swiglu_bwd(x, T, nullptr, 1, T, w13s, H, Is, dh_s, dgu_s, status, st));
-        MOE_TRY(gemm_bf16(dgu_s, T, nullptr, 1, T, w13st, H, 2 * Is, dx_s, status, st));
+        MOE_TRY(gemm_bf16_mn(dgu_s, T, nullptr, 1, T, w13s, H, 2 * Is, 2 * Is, dx_s, status, st));
     }
 
     // input gradient
-    MOE_TRY(launch_unpermute(c, dx_perm, dest_row, dx_s, dx_r, mask, dx, st));
+    MOE_TRY(launch_unpermute(c, dx_perm, dest_pad, dx_s, dx_r, mask, dx, st));
 
-    // weight gradients: each expert's rows as a K range padded to 64 (zero columns)
-    MOE_TRY(launch_padded_offsets(offsets, E, 0, poff, st));
-    MOE_TRY(launch_colmap(offsets, poff, E, A, colmap, st));
-    MOE_TRY(launch_transpose(dy, A, H, H, 0, dyT, rp, 0, 1, colmap, st));
-    MOE_TRY(launch_zero_pad(dyT, H, rp, offsets, poff, E, 0, st));
-    MOE_TRY(launch_transpose(h, A, I, I, 0, hT, rp, 0, 1, colmap, st));
-    MOE_TRY(launch_zero_pad(hT, I, rp, offsets, poff, E, 0, st));
-    MOE_TRY(launch_transpose(dgu, A, 2 * I, 2 * I, 0, dguT, rp, 0, 1, colmap, st));
-    MOE_TRY(launch_zero_pad(dguT, 2 * I, rp, offsets, poff, E, 0, st));
-    MOE_TRY(launch_transpose(x_perm, A, H, H, 0, xpT, rp, 0, 1, colmap, st));
-    MOE_TRY(launch_zero_pad(xpT, H, rp, offsets, poff, E, 0, st));
-    MOE_TRY(gemm_wgrad(dyT, H, hT, I, rp, poff, E, dw2, status, st));
-    MOE_TRY(gemm_wgrad(dguT, 2 * I, xpT, H, rp, poff, E, dw13, status, st));
-
-    // router weights: dW_router = sum_t bf16(dlogits_t)^T x_t
-    MOE_TRY(launch_padded_offsets(nullptr, 1, T, poffT, st));
-    MOE_TRY(launch_transpose(dl_bf, T, ep, ep, 0, dlT, tp, 0, 1, nullptr, st));
-    MOE_TRY(launch_zero_pad(dlT, ep, tp, nullptr, poffT, 1, T, st));
-    MOE_TRY(launch_transpose(x, T, H, H, 0, xT, tp, 0, 1, nullptr, st));
-    MOE_TRY(launch_zero_pad(xT, H, tp, nullptr, poffT, 1, T, st));
-    MOE_TRY(gemm_wgrad(dlT, E, xT, H, tp, poffT, 1, dwr, status, st));
-
+    // weight gradients, operands read in place (MN-major): an expert's K range is its padded
+    // rows; the single-group products take K = T rounded up to 64, the rows past T reading
+    // as zeros
+    MOE_TRY(gemm_wgrad_mn(dy, H, H, h, I, rp, poff, E, dw2, status, st));
+    MOE_TRY(gemm_wgrad_mn(dgu, 2 * I, 2 * I, x_perm, H, rp, poff, E, dw13, status, st));
+    MOE_TRY(launch_padded_offsets(nullptr, 1, T, koffT, st));
+    MOE_TRY(gemm_wgrad_mn(dl_bf, ep, E, x, H, T, koffT, 1, dwr, status, st));
     if (shared) {
-        uint16_t* dysT = at<uint16_t>(ws, L.dysT);
-        uint16_t* hsT = at<uint16_t>(ws, L.hsT);
-        uint16_t* dgusT = at<uint16_t>(ws, L.dgusT);
-        MOE_TRY(launch_transpose(dy_s, T, H, H, 0, dysT, tp, 0, 1, nullptr, st));
-        MOE_TRY(launch_zero_pad(dysT, H, tp, nullptr, poffT, 1, T, st));
-        MOE_TRY(launch_transpose(h_s, T, Is, Is, 0, hsT, tp, 0, 1, nullptr, st));
-        MOE_TRY(launch_zero_pad(hsT, Is, tp, nullptr, poffT, 1, T, st));
-        MOE_TRY(launch_transpose(dgu_s, T, 2 * Is, 2 * Is, 0, dgusT, tp, 0, 1, nullptr, st));
-        MOE_TRY(launch_zero_pad(dgusT, 2 * Is, tp, nullptr, poffT, 1, T, st));
-        MOE_TRY(gemm_wgrad(dysT, H, hsT, Is, tp, poffT, 1, dw2s, status, st));
-        MOE_TRY(gemm_wgrad(dgusT, 2 * Is, xT, H, tp, poffT, 1, dw13s, status, st));
+        MOE_TRY(gemm_wgrad_mn(dy_s, H, H, h_s, Is, T, koffT, 1, dw2s, status, st));
+        MOE_TRY(gemm_wgrad_mn(dgu_s, 2 * Is, 2 * Is, x, H, T, koffT, 1, dw13s, status, st));
     }
     return MOE_OK;
 }

@@ -98,13 +98,14 @@ cudaError_t launch_unpermute(const moe_cfg& c, const uint16_t* rows, const int32
                              uint16_t* dx, cudaStream_t st);
 cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* poff,
                                   cudaStream_t st);
-cudaError_t launch_colmap(const int32_t* off, const int32_t* poff, int G, int64_t rows_bound,
-                          int32_t* col, cudaStream_t st);
-cudaError_t launch_transpose(const uint16_t* in, int64_t R, int F, int64_t ld_in, int64_t in_batch,
-                             uint16_t* out, int64_t ld_out, int64_t out_batch, int batches,
-                             const int32_t* colmap, cudaStream_t st);
-cudaError_t launch_zero_pad(uint16_t* out, int F, int64_t ld_out, const int32_t* off,
-                            const int32_t* poff, int G, int rows, cudaStream_t st);
+// dest_row (dispatch rows) -> rows of the layout whose expert ranges start at poff (each
+// padded to 64 rows): r' = poff[e] + (r - off[e]), e = ids[a]; -1 stays -1
+cudaError_t launch_pad_rows(const int32_t* ids, const int32_t* dest_row, const int32_t* off,
+                            const int32_t* poff, int64_t A, int E, int32_t* dest_pad,
+                            cudaStream_t st);
+// zero rows [poff[g] + n_g, poff[g+1]) of a [rows, cols] bf16 buffer, n_g = off[g+1] - off[g]
+cudaError_t launch_zero_pad_rows(uint16_t* buf, int64_t cols, const int32_t* off,
+                                 const int32_t* poff, int G, cudaStream_t st);
 
 // tensor-core GEMMs (tcgen05 / TMEM / TMA)
 //   EPI_SWIGLU      out[r, c] = bf16(silu(g) * u) of A . B_g^T (gate and up columns paired)
@@ -142,6 +143,9 @@ struct GemmProblem {
     const uint16_t* aux;     // EPI_SWIGLU_BWD: dh [rows, ld_aux] bf16
     int64_t ld_aux;
     const int32_t* k_offsets;  // EPI_WGRAD: device [groups+1] K ranges (multiples of 64)
+    int b_mn;                // B given MN-major, [groups * b_k_rows, n] (K rows of each group,
+    int b_k_rows;            //   N contiguous), read without transposing (EPI_WGRAD: [k, n])
+    int a_mn;                // EPI_WGRAD: A given MN-major, [k, a_rows] (features contiguous)
 };
 
 // the grouped expert products on CTA pairs

@@ -51,9 +51,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Wait for the phase of parity `parity` of `bar` to complete. Gives up (returns false)
-// after about a second, or as soon as another role raised the abort flag.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status, bool honour_abort = true)
+// after about a second, or as soon as another role raised the abort flag. The polling loop
+// is out of line; wait_bounded() below tests the barrier inline first.
+__device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, int32_t* status,
+                                               bool honour_abort)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -70,6 +72,14 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int* abort_flag, int32_t* status,
+                                             bool honour_abort = true)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded_slow(bar, parity, abort_flag, status, honour_abort);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -303,11 +313,30 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
     return d;
 }
 
+// Shared-memory descriptor of an MN-major operand tile with the 128-byte swizzle: TMA boxes
+// of 64 MN-contiguous elements x 64 K rows, one box per 64 MN elements at `mn_box_bytes`
+// apart (leading byte offset); 8-row K groups 1024 bytes apart (stride byte offset). One
+// K=16 step advances the start address by 2048 bytes.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t mn_box_bytes)
+{
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3fffu);
+    d |= (uint64_t)((mn_box_bytes >> 4) & 0x3fffu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t make_idesc(int m, int n)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(m >> 4) << 24);
+}
+// the same with A and/or B MN-major (bits 15 and 16: the operand is transposed)
+__host__ __device__ constexpr uint32_t make_idesc_major(int m, int n, bool a_mn, bool b_mn)
+{
+    return make_idesc(m, n) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
 // bf16 round-to-nearest-even of two floats packed low/high (NaN stays NaN, quieted)

@@ -65,6 +65,7 @@ struct PairArgs {
     int64_t ld_aux;
     int half_out;                // EPI_SWIGLU_BWD: column of the first up gradient
     const float* bias;           // EPI_F32: per-column bias or NULL
+    int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
 };
 
 template <int EPI, int NP>
@@ -129,7 +130,9 @@ __device__ __forceinline__ PairTile decode_wgrad_tile(int t, const PairArgs& a)
     return ti;
 }
 
-template <int EPI, int NP, bool GATHER>
+// MN: operand majorness fixed at compile time -- 0 both K-major, 1 B MN-major, 2 A and B
+// MN-major (the weight-gradient products)
+template <int EPI, int NP, bool GATHER, int MN>
 __global__ void __launch_bounds__(kThreads2, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -138,6 +141,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
     using C = Cfg2<EPI, NP>;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = make_idesc(PM, NP);
+    constexpr uint32_t kIdescBmn = make_idesc_major(PM, NP, false, true);
+    constexpr uint32_t kIdescAB = make_idesc_major(PM, NP, true, true);
     constexpr int kBRows = NP / 2;  // B rows per CTA per stage
 
     extern __shared__ uint8_t smem_raw[];
@@ -244,8 +249,24 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     const uint32_t fb = mapa_shared(full_bar(stage), 0);
                     if (leader) mbar_expect_tx(full_bar(stage), 2 * C::kStageBytes);
                     const int kx = ti.k0 + kb * BK;
-                    tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, kx, arow, fb);
-                    tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kx, brow, fb);
+                    if (MN == 2) {
+                        // this CTA's 128 A features as two 64-feature boxes of 64 K rows
+                        tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, arow, kx, fb);
+                        tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes + 8192u, &tmA,
+                                         arow + 64, kx, fb);
+                    } else {
+                        tma_load_2d_pair(sA0 + (uint32_t)stage * kA2Bytes, &tmA, kx, arow, fb);
+                    }
+                    if (MN >= 1) {
+                        // this CTA's B columns [bcol, bcol + kBRows) of rows g * b_k_rows + kx ..
+                        const int bcol = ti.n * NP + (int)rank * kBRows;
+#pragma unroll
+                        for (int q = 0; q < kBRows / 64; ++q)
+                            tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes + (uint32_t)q * 8192u,
+                                             &tmB, bcol + 64 * q, ti.g * args.b_k_rows + kx, fb);
+                    } else {
+                        tma_load_2d_pair(sB0 + (uint32_t)stage * C::kBBytes, &tmB, kx, brow, fb);
+                    }
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) {
@@ -373,12 +394,19 @@ __global__ void __launch_bounds__(kThreads2, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = sw128_desc(sA0 + (uint32_t)stage * kA2Bytes);
-                    const uint64_t bd = sw128_desc(sB0 + (uint32_t)stage * C::kBBytes);
+                    const uint32_t sa = sA0 + (uint32_t)stage * kA2Bytes;
+                    const uint32_t sb = sB0 + (uint32_t)stage * C::kBBytes;
+                    // K-major operand: +32 bytes per K=16 step inside the swizzle row;
+                    // MN-major operand: +2048 bytes (16 K rows of 128 bytes)
+                    const uint64_t ad = MN == 2 ? sw128_mn_desc(sa, 8192u) : sw128_desc(sa);
+                    const uint64_t bd = MN >= 1 ? sw128_mn_desc(sb, 8192u) : sw128_desc(sb);
+                    constexpr uint64_t astep = MN == 2 ? 128u : 2u;
+                    constexpr uint64_t bstep = MN >= 1 ? 128u : 2u;
+                    constexpr uint32_t idesc = MN == 2 ? kIdescAB : (MN == 1 ? kIdescBmn : kIdesc);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
-                                      kIdesc, (kb | k) != 0 ? 1u : 0u);
+                        mma_bf16_pair(d_tmem, ad + astep * (uint64_t)k, bd + bstep * (uint64_t)k,
+                                      idesc, (kb | k) != 0 ? 1u : 0u);
                     mma_commit_pair_mc(empty_bar(stage), kPairMask);
                     if (++stage == S) {
                         stage = 0;
@@ -582,11 +610,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
     }
 }
 
-template <int EPI, int NP, bool GATHER>
+template <int EPI, int NP, bool GATHER, int MN = 0>
 cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
 {
     using C = Cfg2<EPI, NP>;
-    auto kernel = tc_gemm_pair_kernel<EPI, NP, GATHER>;
+    auto kernel = tc_gemm_pair_kernel<EPI, NP, GATHER, MN>;
     const int groups = (p.offsets || EPI == EPI_WGRAD) ? p.groups : 1;
     const size_t smem = C::smem_bytes(groups);
     int dev = 0;
@@ -629,10 +657,22 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
     CUtensorMap ma, mb, mo;
     const bool wgrad = (EPI == EPI_WGRAD);
-    if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) return cudaErrorInvalidValue;
-    if (!make_map(&mb, p.b, wgrad ? (int64_t)p.n : (int64_t)groups * p.b_rows_per_group, p.k,
-                  NP / 2))
+    if (p.a_mn) {
+        // [k, a_rows] with the features contiguous: boxes of 64 features x 64 K rows
+        if (!wgrad || p.a_rows % 8 != 0) return cudaErrorInvalidValue;
+        if (!make_map(&ma, p.a, p.k, p.a_rows, 64)) return cudaErrorInvalidValue;
+    } else if (!make_map(&ma, p.a, p.a_rows, p.k, HM)) {
         return cudaErrorInvalidValue;
+    }
+    if (p.b_mn) {
+        // [groups * b_k_rows, n] (EPI_WGRAD: [k, n]) with N contiguous: 64 x 64 boxes
+        if (p.n % 64 != 0 || (!wgrad && p.b_k_rows < 1)) return cudaErrorInvalidValue;
+        if (!make_map(&mb, p.b, wgrad ? (int64_t)p.k : (int64_t)groups * p.b_k_rows, p.n, 64))
+            return cudaErrorInvalidValue;
+    } else if (!make_map(&mb, p.b, wgrad ? (int64_t)p.n : (int64_t)groups * p.b_rows_per_group, p.k,
+                         NP / 2)) {
+        return cudaErrorInvalidValue;
+    }
     if (wgrad || EPI == EPI_F32) {
         mo = mb;  // fp32 rows are stored from registers; the store map is not used
     } else {
@@ -655,6 +695,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.ld_aux = p.ld_aux;
     a.half_out = (EPI == EPI_SWIGLU_BWD) ? p.n : 0;
     a.bias = p.bias;
+    a.b_k_rows = wgrad ? 0 : p.b_k_rows;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;
@@ -674,29 +715,46 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
 
 cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st)
 {
-    if (p.k % BK != 0) return cudaErrorInvalidValue;
+    // K-major operands are read in 64-wide k-blocks; MN-major weight-gradient operands have
+    // any number of K rows (the last block reads zeros past the end)
+    if (!(p.epilogue == EPI_WGRAD && p.a_mn && p.b_mn) && p.k % BK != 0)
+        return cudaErrorInvalidValue;
     if (p.epilogue == EPI_SWIGLU) {
         if (p.n % 128 != 0) return cudaErrorInvalidValue;
         if (p.gather_rows) return launch_pair_variant<EPI_SWIGLU, 256, true>(p, st);
         return launch_pair_variant<EPI_SWIGLU, 256, false>(p, st);
     }
     if (p.gather_rows) return cudaErrorInvalidValue;
+    if (p.b_mn && p.epilogue != EPI_BF16 && p.epilogue != EPI_F32 && p.epilogue != EPI_WGRAD)
+        return cudaErrorInvalidValue;
     if (p.epilogue == EPI_SWIGLU_BWD) {
         if (p.n % 128 != 0 || p.aux == nullptr) return cudaErrorInvalidValue;
         return launch_pair_variant<EPI_SWIGLU_BWD, 256, false>(p, st);
     }
     if (p.epilogue == EPI_WGRAD) {
         if (p.k_offsets == nullptr || p.rows < 1) return cudaErrorInvalidValue;
+        if (p.a_mn != p.b_mn) return cudaErrorInvalidValue;
+        if (p.a_mn) {
+            if (p.n % 256 == 0) return launch_pair_variant<EPI_WGRAD, 256, false, 2>(p, st);
+            if (p.n % 128 == 0) return launch_pair_variant<EPI_WGRAD, 128, false, 2>(p, st);
+            return cudaErrorInvalidValue;
+        }
         if (p.n % 256 == 0) return launch_pair_variant<EPI_WGRAD, 256, false>(p, st);
         if (p.n % 128 == 0) return launch_pair_variant<EPI_WGRAD, 128, false>(p, st);
         return cudaErrorInvalidValue;
     }
     if (p.epilogue == EPI_F32) {
+        if (p.b_mn) return cudaErrorInvalidValue;
         if (p.n % 256 == 0) return launch_pair_variant<EPI_F32, 256, false>(p, st);
         if (p.n % 128 == 0) return launch_pair_variant<EPI_F32, 128, false>(p, st);
         return cudaErrorInvalidValue;
     }
     if (p.epilogue == EPI_BF16) {
+        if (p.b_mn) {
+            if (p.n % 256 == 0) return launch_pair_variant<EPI_BF16, 256, false, 1>(p, st);
+            if (p.n % 128 == 0) return launch_pair_variant<EPI_BF16, 128, false, 1>(p, st);
+            return cudaErrorInvalidValue;
+        }
         if (p.n % 256 == 0) return launch_pair_variant<EPI_BF16, 256, false>(p, st);
         if (p.n % 128 == 0) return launch_pair_variant<EPI_BF16, 128, false>(p, st);
     }
