@@ -291,6 +291,20 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, tflops, reps=20):
                                b["topk_ids"], b["topk_w"], dout, w13_s=w.get("w13_s"),
                                w2_s=w.get("w2_s"), ws=ws, check=False)
     ms_b = loop(bwd)
+    # the training pair: moe_forward_train leaves the intermediates, the backward reuses them
+    moe.forward_train(cfg, x, w["w_router"], w["w13"], w["w2"], ws, w13_s=w.get("w13_s"),
+                      w2_s=w.get("w2_s"), logit_bias=w.get("logit_bias"),
+                      sel_bias=w.get("sel_bias"))
+    bwd_saved = lambda: moe.backward(cfg, x, w["w_router"], w["w13"], w["w2"],  # noqa: E731
+                                     b["logits"], b["topk_ids"], b["topk_w"], dout,
+                                     w13_s=w.get("w13_s"), w2_s=w.get("w2_s"), ws=ws,
+                                     saved=True, check=False)
+    ms_bs = loop(bwd_saved)
+    fwd_train = lambda: moe.forward_train(cfg, x, w["w_router"], w["w13"], w["w2"], ws,  # noqa: E731
+                                          w13_s=w.get("w13_s"), w2_s=w.get("w2_s"),
+                                          logit_bias=w.get("logit_bias"),
+                                          sel_bias=w.get("sel_bias"), check=False)
+    ms_ft = loop(fwd_train)
     rows = int(offsets[-1].item())
     I, Is = cfg.I, cfg.I_shared
     # algorithmic: dh, dx rows, dW2, dW13 (12 H I per routed row), router dx and dW, shared
@@ -316,7 +330,11 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, tflops, reps=20):
                      "frac_bf16_sustained": bwd_flops / (ms_b * 1e-3) / 1e12 / tflops,
                      "executed_flops_with_recompute": bwd_flops + recompute_flops,
                      "call": "moe_backward (dx, dW13, dW2, dW_router; forward intermediates "
-                             "recomputed)"},
+                             "recomputed)",
+                     "ms_with_saved_intermediates": ms_bs,
+                     "frac_bf16_sustained_saved": bwd_flops / (ms_bs * 1e-3) / 1e12 / tflops,
+                     "forward_train_ms": ms_ft,
+                     "train_step_ms": ms_ft + ms_bs},
         "timing": f"CUDA events, {reps} back-to-back launches each, inputs of one bench step",
     }
 

@@ -65,7 +65,8 @@ SIGNATURES = {
     "moe_forward": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          _SZ, _P, _P]),
     "moe_router_stats": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
-    "moe_backward": (_I, [_CFG] + [_P] * 21 + [_SZ, _P]),
+    "moe_backward": (_I, [_CFG] + [_P] * 19 + [_I, _P, _P, _SZ, _P]),
+    "moe_forward_train": (_I, [_CFG] + [_P] * 15 + [_SZ, _P]),
     "moe_forward_host_workspace_bytes": (_SZ, [_CFG, _I]),
     "moe_forward_host": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),

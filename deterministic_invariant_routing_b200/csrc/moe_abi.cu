@@ -406,7 +406,7 @@ size_t pad64(size_t v) { return (v + 63) / 64 * 64; }
 // form whole 64-row K blocks of the weight-gradient products.
 struct BwdLayout {
     size_t offsets, perm_token, dest_row, dest_pad, poff, perm_ws, x_perm, h, y, dy, dh, dgu,
-        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, dh_s, dgu_s, dx_s, dy_s, total;
+        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, dh_s, dgu_s, dx_s, dy_s, y_s, total;
     int64_t rp, e_pad;
 };
 
@@ -446,6 +446,7 @@ BwdLayout bwd_layout(const moe_cfg& c)
     L.dgu_s = take(T * 2 * Is * 2);
     L.dx_s = take(Is ? T * H * 2 : 0);
     L.dy_s = take(Is ? T * H * 2 : 0);
+    L.y_s = take(Is ? T * H * 2 : 0);
     L.total = off;
     return L;
 }
@@ -480,15 +481,46 @@ cudaError_t gemm_wgrad_mn(const uint16_t* a, int64_t a_cols, int m, const uint16
         if (rc_ != MOE_OK) return rc_;                  \
     } while (0)
 
+// Dispatch into the padded layout and the expert intermediates the backward reuses:
+// offsets, dest_pad, poff, x_perm (padding rows zero), h, y, and the shared expert's h_s.
+// moe_forward_train leaves them in the workspace; moe_backward recomputes them otherwise
+// (the same products: a row's bits do not depend on where it sits).
+int train_intermediates(const moe_cfg& c, const uint16_t* x, const int32_t* ids,
+                        const uint16_t* w13, const uint16_t* w2, const uint16_t* w13s,
+                        int32_t* status, void* ws, cudaStream_t st)
+{
+    const BwdLayout L = bwd_layout(c);
+    const int64_t A = (int64_t)c.T * c.K;
+    const int H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
+    const int64_t rp = L.rp;
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* dest_row = at<int32_t>(ws, L.dest_row);
+    int32_t* dest_pad = at<int32_t>(ws, L.dest_pad);
+    int32_t* poff = at<int32_t>(ws, L.poff);
+    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+    uint16_t* h = at<uint16_t>(ws, L.h);
+    MOE_TRY(launch_permute(c, ids, offsets, at<int32_t>(ws, L.perm_token), dest_row, status,
+                           at<void>(ws, L.perm_ws), st));
+    MOE_TRY(launch_padded_offsets(offsets, E, 0, poff, st));
+    MOE_TRY(launch_pad_rows(ids, dest_row, offsets, poff, A, E, dest_pad, st));
+    MOE_TRY(launch_zero_pad_rows(x_perm, H, offsets, poff, E, st));
+    MOE_TRY(launch_gather_rows(c, x, dest_pad, x_perm, st));
+    MOE_TRY(gate_up(x_perm, rp, nullptr, rp, poff, E, 0, w13, H, I, h, status, st));
+    MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, at<uint16_t>(ws, L.y), status, st));
+    if (Is > 0)
+        MOE_TRY(gate_up(x, T, nullptr, T, nullptr, 1, T, w13s, H, Is, at<uint16_t>(ws, L.h_s),
+                        status, st));
+    return MOE_OK;
+}
+
 int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const uint8_t* mask,
                   const uint16_t* w13, const uint16_t* w2, const uint16_t* w13s,
                   const uint16_t* w2s, const float* logits, const int32_t* ids,
                   const float* topk_w, const uint16_t* dout, uint16_t* dx, float* dwr,
                   float* dw13, float* dw2, float* dw13s, float* dw2s, float* d_topk_w,
-                  float* dlogits, int32_t* status, void* ws, cudaStream_t st)
+                  float* dlogits, int saved, int32_t* status, void* ws, cudaStream_t st)
 {
     const BwdLayout L = bwd_layout(c);
-    const int64_t A = (int64_t)c.T * c.K;
     const int H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
     const int ep = (int)L.e_pad;
     const int64_t rp = L.rp;
@@ -510,18 +542,13 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     uint16_t* dx_r = at<uint16_t>(ws, L.dx_r);
     int32_t* koffT = at<int32_t>(ws, L.koffT);
 
-    // dispatch, then the padded row layout (expert ranges at poff, padding rows zero)
-    MOE_TRY(launch_permute(c, ids, offsets, at<int32_t>(ws, L.perm_token), dest_row, status,
-                           at<void>(ws, L.perm_ws), st));
-    MOE_TRY(launch_padded_offsets(offsets, E, 0, poff, st));
-    MOE_TRY(launch_pad_rows(ids, dest_row, offsets, poff, A, E, dest_pad, st));
-    MOE_TRY(launch_zero_pad_rows(x_perm, H, offsets, poff, E, st));
+    // dispatch into the padded layout and the forward intermediates (padding rows give
+    // h = 0, y = 0), unless moe_forward_train left them in the workspace
+    if (!saved) {
+        const int rc = train_intermediates(c, x, ids, w13, w2, w13s, status, ws, st);
+        if (rc != MOE_OK) return rc;
+    }
     MOE_TRY(launch_zero_pad_rows(dy, H, offsets, poff, E, st));
-    MOE_TRY(launch_gather_rows(c, x, dest_pad, x_perm, st));
-    // the forward intermediates recomputed (the same products: a row's bits do not depend on
-    // where it sits); padding rows give h = 0, y = 0
-    MOE_TRY(gate_up(x_perm, rp, nullptr, rp, poff, E, 0, w13, H, I, h, status, st));
-    MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, y, status, st));
 
     // combine backward: routing-weight gradients and the expert-output gradients
     uint16_t* dy_s = shared ? at<uint16_t>(ws, L.dy_s) : nullptr;
@@ -545,7 +572,6 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
         uint16_t* dh_s = at<uint16_t>(ws, L.dh_s);
         dgu_s = at<uint16_t>(ws, L.dgu_s);
         dx_s = at<uint16_t>(ws, L.dx_s);
-        MOE_TRY(gate_up(x, T, nullptr, T, nullptr, 1, T, w13s, H, Is, h_s, status, st));
         MOE_TRY(gemm_bf16_mn(dy_s, T, nullptr, 1, T, w2s, Is, H, H, dh_s, status, st));
         MOE_TRY(gemm_swiglu_bwd(x, T, nullptr, 1, T, w13s, H, Is, dh_s, dgu_s, status, st));
         MOE_TRY(gemm_bf16_mn(dgu_s, T, nullptr, 1, T, w13s, H, 2 * Is, 2 * Is, dx_s, status, st));
@@ -577,7 +603,7 @@ using namespace moe;
 
 extern "C" {
 
-MOE_API int moe_abi_version(void) { return 102; }
+MOE_API int moe_abi_version(void) { return 103; }
 
 MOE_API const char* moe_status_string(int code)
 {
@@ -845,12 +871,13 @@ MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* 
                          const uint16_t* w13_s, const uint16_t* w2_s, const float* logits,
                          const int32_t* topk_ids, const float* topk_w, const uint16_t* dout,
                          uint16_t* dx, float* dw_router, float* dw13, float* dw2, float* dw13_s,
-                         float* dw2_s, float* d_topk_w, float* dlogits, int32_t* status,
-                         void* ws, size_t ws_bytes, void* stream)
+                         float* dw2_s, float* d_topk_w, float* dlogits, int saved,
+                         int32_t* status, void* ws, size_t ws_bytes, void* stream)
 {
     int rc = check_cfg(cfg);
     if (rc != MOE_OK) return rc;
     const moe_cfg& c = *cfg;
+    if (saved != 0 && saved != 1) return MOE_ERR_ARG;
     const void* need[] = {w_router, w13, w2, dw_router, dw13, dw2, status};
     for (const void* q : need)
         if (q == nullptr) return MOE_ERR_ARG;
@@ -887,7 +914,44 @@ MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* 
     }
     return backward_impl(c, x, w_router, token_mask, w13, w2, w13_s, w2_s, logits, topk_ids,
                          topk_w, dout, dx, dw_router, dw13, dw2, dw13_s, dw2_s, d_topk_w, dlogits,
-                         status, ws, st);
+                         saved, status, ws, st);
+}
+
+MOE_API int moe_forward_train(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                              const float* logit_bias, const float* sel_bias,
+                              const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                              const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out,
+                              float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                              void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_forward_args(cfg, x, w_router, w13, w2, w13_s, w2_s, out, status);
+    if (rc != MOE_OK) return rc;
+    const moe_cfg& c = *cfg;
+    if (c.T > 0 && (logits == nullptr || topk_ids == nullptr || topk_w == nullptr))
+        return MOE_ERR_ARG;
+    if ((logits && !aligned16(logits)) || (topk_ids && !aligned16(topk_ids)) ||
+        (topk_w && !aligned16(topk_w)))
+        return MOE_ERR_ARG;
+    const BwdLayout L = bwd_layout(c);
+    if (ws == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (c.T == 0) return MOE_OK;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    if ((rc = router_and_route(c, x, w_router, logit_bias, sel_bias, token_mask, logits, topk_ids,
+                               topk_w, status, nullptr, st)) != MOE_OK)
+        return rc;
+    if ((rc = train_intermediates(c, x, topk_ids, w13, w2, w13_s, status, ws, st)) != MOE_OK)
+        return rc;
+    uint16_t* y_s = nullptr;
+    if (c.I_shared > 0) {
+        y_s = at<uint16_t>(ws, L.y_s);
+        if ((rc = cuda_rc(down(at<uint16_t>(ws, L.h_s), c.T, nullptr, 1, c.T, w2_s, c.H,
+                               c.I_shared, y_s, status, st))) != MOE_OK)
+            return rc;
+    }
+    return cuda_rc(launch_combine(c, at<uint16_t>(ws, L.y), topk_w, at<int32_t>(ws, L.dest_pad),
+                                  y_s, token_mask, out, st));
 }
 
 }  // extern "C"

@@ -242,13 +242,55 @@ def router_stats(cfg: Config, logits, offsets, token_mask=None):
 
 # ------------------------------------------------------------------ backward
 
+def backward_workspace(cfg: Config, dev) -> torch.Tensor:
+    """A workspace for forward_train() + backward(saved=True) (or backward alone)."""
+    return _ws(workspace_bytes(cfg, N.MOE_STAGE_BACKWARD), dev, None)
+
+
+def forward_train(cfg: Config, x, w_router, w13, w2, ws, logit_bias=None, sel_bias=None,
+                  token_mask=None, w13_s=None, w2_s=None, status=None, check: bool = True):
+    """The forward of a training step (moe_forward_train): the same output as forward(), and
+    the intermediates the backward needs left in `ws` (backward_workspace()). Returns
+    (out [T,H] bf16, {logits, topk_ids, topk_w}); then backward(..., ws=ws, saved=True)."""
+    dev = x.device
+    T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
+    _need(x, "x", torch.bfloat16, (T, H), dev)
+    _need(w_router, "w_router", torch.bfloat16, (E, H), dev)
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H), dev)
+    _need(w2, "w2", torch.bfloat16, (E, H, I), dev)
+    _opt(logit_bias, "logit_bias", torch.float32, (E,), dev)
+    _opt(sel_bias, "sel_bias", torch.float32, (E,), dev)
+    _opt(token_mask, "token_mask", torch.uint8, (T,), dev)
+    if Is:
+        _need(w13_s, "w13_s", torch.bfloat16, (2 * Is, H), dev)
+        _need(w2_s, "w2_s", torch.bfloat16, (H, Is), dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    b = {"logits": torch.empty(T, E, dtype=torch.float32, device=dev),
+         "topk_ids": torch.empty(T, K, dtype=torch.int32, device=dev),
+         "topk_w": torch.empty(T, K, dtype=torch.float32, device=dev)}
+    nbytes = workspace_bytes(cfg, N.MOE_STAGE_BACKWARD)
+    ws = _ws(nbytes, dev, ws)
+    st = new_status(dev) if status is None else status
+    _rc(N.load().moe_forward_train(ctypes.byref(cfg.c()), _p(x), _p(w_router), _p(logit_bias),
+                                   _p(sel_bias), _p(token_mask), _p(w13), _p(w2), _p(w13_s),
+                                   _p(w2_s), _p(out), _p(b["logits"]), _p(b["topk_ids"]),
+                                   _p(b["topk_w"]), _p(st), _p(ws), nbytes, _stream(dev)),
+        "moe_forward_train")
+    if check:
+        check_status(st)
+    return out, b
+
+
 def backward(cfg: Config, x, w_router, w13, w2, logits, topk_ids, topk_w, dout, token_mask=None,
              w13_s=None, w2_s=None, ws=None, status=None, keep: bool = False,
-             check: bool = True) -> dict:
+             saved: bool = False, check: bool = True) -> dict:
     """Gradients of sum(dout * out) of the layer for the forward's routes (moe_backward):
     {dx [T,H] bf16, dw_router [E,H], dw13 [E,2I,H], dw2 [E,H,I] fp32 (+ dw13_s, dw2_s with a
     shared expert)}; keep=True adds d_topk_w [T,K] and dlogits [T,E] (fp32).
-    logits, topk_ids, topk_w: as forward(keep=True) returned them."""
+    logits, topk_ids, topk_w: as forward(keep=True) or forward_train() returned them.
+    saved=True: ws holds forward_train()'s intermediates for the same inputs (no recompute)."""
+    if saved and ws is None:
+        raise MoeError("saved=True needs the workspace forward_train() wrote")
     dev = x.device
     T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
     _need(x, "x", torch.bfloat16, (T, H), dev)
@@ -279,8 +321,8 @@ def backward(cfg: Config, x, w_router, w13, w2, logits, topk_ids, topk_w, dout, 
                               _p(w13), _p(w2), _p(w13_s), _p(w2_s), _p(logits), _p(topk_ids),
                               _p(topk_w), _p(dout), _p(g["dx"]), _p(g["dw_router"]),
                               _p(g["dw13"]), _p(g["dw2"]), _p(g["dw13_s"]), _p(g["dw2_s"]),
-                              _p(g.get("d_topk_w")), _p(g.get("dlogits")), _p(st), _p(ws),
-                              nbytes, _stream(dev)), "moe_backward")
+                              _p(g.get("d_topk_w")), _p(g.get("dlogits")), int(bool(saved)),
+                              _p(st), _p(ws), nbytes, _stream(dev)), "moe_backward")
     if check:
         check_status(st)
     return g

@@ -345,6 +345,8 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
  *      for masked tokens;
  *    dW = sum over an expert's rows, ascending, of dy^T h / [dg|du]^T x (fp32 accumulation
  *      on the tensor cores, bf16 operands); dW_router = sum_t bf16(dlogits_t)^T x_t.
+ *  saved  0: the forward intermediates are recomputed from x; 1: `ws` holds those that
+ *         moe_forward_train wrote for the same cfg, inputs and routes (not checked).
  *  ws  moe_workspace_bytes(cfg, MOE_STAGE_BACKWARD) bytes.
  */
 MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
@@ -352,8 +354,22 @@ MOE_API int moe_backward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* 
                          const uint16_t* w13_s, const uint16_t* w2_s, const float* logits,
                          const int32_t* topk_ids, const float* topk_w, const uint16_t* dout,
                          uint16_t* dx, float* dw_router, float* dw13, float* dw2, float* dw13_s,
-                         float* dw2_s, float* d_topk_w, float* dlogits, int32_t* status,
-                         void* ws, size_t ws_bytes, void* stream);
+                         float* dw2_s, float* d_topk_w, float* dlogits, int saved,
+                         int32_t* status, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The forward of a training step: the same output bits as moe_forward, and the dispatch
+ * and expert intermediates the backward needs left in `ws` (the backward's workspace,
+ * moe_workspace_bytes(cfg, MOE_STAGE_BACKWARD) bytes), so that moe_backward with saved = 1
+ * on the same ws, cfg, inputs and routes skips recomputing them. logits, topk_ids and topk_w
+ * (device outputs, required) are the routes the backward takes.
+ */
+MOE_API int moe_forward_train(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
+                              const float* logit_bias, const float* sel_bias,
+                              const uint8_t* token_mask, const uint16_t* w13, const uint16_t* w2,
+                              const uint16_t* w13_s, const uint16_t* w2_s, uint16_t* out,
+                              float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /* Text of a return code. */
 MOE_API const char* moe_status_string(int code);

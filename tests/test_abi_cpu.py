@@ -42,7 +42,7 @@ def test_status_strings(lib):
     assert N.status_string(0) == "ok"
     for code in (-1, -2, -3, -4, -5, -6):
         assert N.status_string(code) != "unknown status"
-    assert lib.moe_abi_version() == 102
+    assert lib.moe_abi_version() == 103
 
 
 GOOD = dict(T=64, H=128, E=8, K=2, I=256)

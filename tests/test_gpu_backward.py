@@ -165,3 +165,30 @@ def test_backward_zero_tokens_gives_zero_weight_gradients():
                      e(0, s.K, device=DEV), e(0, s.H, dtype=torch.bfloat16, device=DEV))
     torch.cuda.synchronize()
     assert not g["dw13"].any() and not g["dw2"].any() and not g["dw_router"].any()
+
+
+@pytest.mark.parametrize("name,T,keep", [("qwen3_30b_a3b", 300, 0.8), ("dsv_sigmoid", 64, None)])
+def test_forward_train_and_saved_backward_equal_the_plain_calls(name, T, keep):
+    """moe_forward_train gives moe_forward's bits and leaves the intermediates; the backward
+    reusing them gives the recomputing backward's bits, for every output."""
+    s, d, cfg = layer(name, T)
+    mask = None if keep is None else synthetic.random_mask(T, keep, 5).to(DEV)
+    kw = dict(logit_bias=d["logit_bias"], sel_bias=d["sel_bias"], token_mask=mask,
+              w13_s=d["w13_s"], w2_s=d["w2_s"])
+    out, b = moe.forward(cfg, d["x"], d["w_router"], d["w13"], d["w2"], keep=True, **kw)
+    ws = moe.backward_workspace(cfg, DEV)
+    out_t, bt = moe.forward_train(cfg, d["x"], d["w_router"], d["w13"], d["w2"], ws, **kw)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(out_t.cpu()), bits(out.cpu()))
+    for k in ("logits", "topk_ids", "topk_w"):
+        assert np.array_equal(bits(bt[k].cpu()), bits(b[k].cpu())), k
+    dout = synthetic.normal_bf16(T, s.H, 1.0, 7, "fill").to(DEV)
+    args = (cfg, d["x"], d["w_router"], d["w13"], d["w2"], bt["logits"], bt["topk_ids"],
+            bt["topk_w"], dout)
+    g0 = moe.backward(*args, token_mask=mask, w13_s=d["w13_s"], w2_s=d["w2_s"], keep=True)
+    g1 = moe.backward(*args, token_mask=mask, w13_s=d["w13_s"], w2_s=d["w2_s"], keep=True,
+                      ws=ws, saved=True)
+    torch.cuda.synchronize()
+    for k, v in g0.items():
+        if v is not None:
+            assert np.array_equal(bits(g1[k].cpu()), bits(v.cpu())), k
