@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t armed = 0, armed_phase = 0;
+            const uint32_t fb0 = mapa_shared(full_bar(0), 0);  // the leader's full[0]
             for (int t = cluster; t < total && !*abort_flag; t += nclusters) {
                 const PairTile ti = decode(t);
                 const int arow = (int)ti.row0 + (int)rank * HM;
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = mapa_shared(full_bar(stage), 0);
+                    const uint32_t fb = fb0 + 8u * (uint32_t)stage;
                     if (leader) mbar_expect_tx(full_bar(stage), 2 * C::kStageBytes);
                     const int kx = ti.k0 + kb * BK;
                     if (MN == 2) {
@@ -376,6 +377,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------------------------------------------------- MMA issuer
+            // K-major operand: +32 bytes per K=16 step inside the swizzle row; MN-major
+            // operand: +2048 bytes (16 K rows of 128 bytes)
+            const uint64_t ad0 = MN == 2 ? sw128_mn_desc(sA0, 8192u) : sw128_desc(sA0);
+            const uint64_t bd0 = MN >= 1 ? sw128_mn_desc(sB0, 8192u) : sw128_desc(sB0);
+            constexpr uint64_t astep = MN == 2 ? 128u : 2u;
+            constexpr uint64_t bstep = MN >= 1 ? 128u : 2u;
+            constexpr uint32_t idesc = MN == 2 ? kIdescAB : (MN == 1 ? kIdescBmn : kIdesc);
             int stage = 0;
             uint32_t phase = 0;
             int i = 0;
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NP);
-                const int kbs = decode(t).kbs;
+                const int kbs = kWgrad ? decode(t).kbs : args.k_blocks;
                 bool ok = true;
                 for (int kb = 0; kb < kbs; ++kb) {
                     if (!wait_bounded(full_bar(stage), phase, abort_flag, args.status)) {
@@ -394,15 +402,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = sA0 + (uint32_t)stage * kA2Bytes;
-                    const uint32_t sb = sB0 + (uint32_t)stage * C::kBBytes;
-                    // K-major operand: +32 bytes per K=16 step inside the swizzle row;
-                    // MN-major operand: +2048 bytes (16 K rows of 128 bytes)
-                    const uint64_t ad = MN == 2 ? sw128_mn_desc(sa, 8192u) : sw128_desc(sa);
-                    const uint64_t bd = MN >= 1 ? sw128_mn_desc(sb, 8192u) : sw128_desc(sb);
-                    constexpr uint64_t astep = MN == 2 ? 128u : 2u;
-                    constexpr uint64_t bstep = MN >= 1 ? 128u : 2u;
-                    constexpr uint32_t idesc = MN == 2 ? kIdescAB : (MN == 1 ? kIdescBmn : kIdesc);
+                    // stage descriptors: the stage-0 ones plus the stage offset (16-byte units)
+                    const uint64_t ad = ad0 + (uint64_t)((uint32_t)stage * (kA2Bytes >> 4));
+                    const uint64_t bd = bd0 + (uint64_t)((uint32_t)stage * (C::kBBytes >> 4));
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
                         mma_bf16_pair(d_tmem, ad + astep * (uint64_t)k, bd + bstep * (uint64_t)k,
