@@ -447,7 +447,7 @@ def main():
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
                 "ms_per_step": ms_e2e, "chunk_tokens": a.e2e_chunk,
                 "call": "moe_forward_host (pinned host in/out, copies overlapped)"},
-        "gpu_launches": K * (9 + (2 if s.I_shared else 0)),
+        "gpu_launches": K * (10 + (3 if s.I_shared else 0)),
         "clocks": clocks,
     }
     if not a.no_extras:

@@ -66,6 +66,8 @@ struct PairArgs {
     int half_out;                // EPI_SWIGLU_BWD: column of the first up gradient
     const float* bias;           // EPI_F32: per-column bias or NULL
     int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
+    int skip_tails;              // leave each group's last rows to the 1-SM tail kernel when
+                                 // they fit one CTA (at most 128 past the last full tile)
 };
 
 template <int EPI, int NP>
@@ -193,11 +195,14 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const int per = (G + 31) / 32;
         const int beg = lane * per < G ? lane * per : G;
         const int end = beg + per < G ? beg + per : G;
+        auto tiles_of = [&](int n) -> int {
+            return args.skip_tails ? n / PM + (n % PM > HM ? 1 : 0) : (n + PM - 1) / PM;
+        };
         int sum = 0;
         for (int g = beg; g < end; ++g) {
             const int r0 = row_off(g);
             offs[g] = r0;
-            sum += (row_off(g + 1) - r0 + PM - 1) / PM;
+            sum += tiles_of(row_off(g + 1) - r0);
         }
         if (lane == 0) offs[G] = row_off(G);
         int incl = sum;
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         int run = incl - sum;
         for (int g = beg; g < end; ++g) {
             prefix[g] = run;
-            run += (row_off(g + 1) - row_off(g) + PM - 1) / PM;
+            run += tiles_of(row_off(g + 1) - row_off(g));
         }
         if (lane == 31) prefix[G] = incl;
     }
@@ -698,6 +703,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.half_out = (EPI == EPI_SWIGLU_BWD) ? p.n : 0;
     a.bias = p.bias;
     a.b_k_rows = wgrad ? 0 : p.b_k_rows;
+    a.skip_tails = p.skip_tails;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;
