@@ -244,12 +244,14 @@ cudaError_t gemm_bf16_mn(const uint16_t* a, int64_t a_rows, const int32_t* offse
 
 // the gate/up product recomputed with the SwiGLU backward in its epilogue:
 // dgu[r] = [dh * u * silu'(g) | dh * silu(g)] (bf16, 2I columns)
-cudaError_t gemm_swiglu_bwd(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
-                            int rows, const uint16_t* w13, int H, int I, const uint16_t* dh,
-                            uint16_t* dgu, int32_t* status, cudaStream_t st)
+// gate_up + SwiGLU over grouped rows (CTA pairs only) that also keeps the fp32 gate and up
+// values: gu[r] = [a_r . W1g^T | a_r . W1u^T], row stride 2 I
+cudaError_t gate_up_save(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                         int rows, const uint16_t* w13, int H, int I, uint16_t* h, float* gu,
+                         int32_t* status, cudaStream_t st)
 {
     GemmProblem p{};
-    p.epilogue = EPI_SWIGLU_BWD;
+    p.epilogue = EPI_SWIGLU_SAVE;
     p.a = a;
     p.a_rows = a_rows;
     p.a_rows_total = a_rows;
@@ -260,10 +262,38 @@ cudaError_t gemm_swiglu_bwd(const uint16_t* a, int64_t a_rows, const int32_t* of
     p.groups = groups;
     p.offsets = offsets;
     p.rows = rows;
+    p.out = h;
+    p.ldo = I;
+    p.gu = gu;
+    p.ld_gu = 2 * (int64_t)I;
+    p.status = status;
+    return launch_tc_gemm_pair(p, st);
+}
+
+// dgu = SwiGLU backward of dh = a . W2 (W2 [groups, H, I] read MN-major), dh kept in fp32,
+// with the gate and up values gu that gate_up_save kept: dgu [rows, 2 I] bf16
+cudaError_t gemm_dswiglu(const uint16_t* a, int64_t a_rows, const int32_t* offsets, int groups,
+                         int rows, const uint16_t* w2, int I, int H, const float* gu,
+                         uint16_t* dgu, int32_t* status, cudaStream_t st)
+{
+    GemmProblem p{};
+    p.epilogue = EPI_DSWIGLU;
+    p.a = a;
+    p.a_rows = a_rows;
+    p.a_rows_total = a_rows;
+    p.b = w2;
+    p.b_rows_per_group = I;
+    p.b_mn = 1;
+    p.b_k_rows = H;
+    p.k = H;
+    p.n = I;
+    p.groups = groups;
+    p.offsets = offsets;
+    p.rows = rows;
     p.out = dgu;
-    p.ldo = 2 * I;
-    p.aux = dh;
-    p.ld_aux = I;
+    p.ldo = 2 * (int64_t)I;
+    p.gu = const_cast<float*>(gu);
+    p.ld_gu = 2 * (int64_t)I;
     p.status = status;
     return launch_tc_gemm_pair(p, st);
 }
@@ -413,8 +443,8 @@ size_t pad64(size_t v) { return (v + 63) / 64 * 64; }
 // poff[e] (its count rounded up to 64, the padding rows zero), so that every expert's rows
 // form whole 64-row K blocks of the weight-gradient products.
 struct BwdLayout {
-    size_t offsets, perm_token, dest_row, dest_pad, poff, perm_ws, x_perm, h, y, dy, dh, dgu,
-        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, dh_s, dgu_s, dx_s, dy_s, y_s, total;
+    size_t offsets, perm_token, dest_row, dest_pad, poff, perm_ws, x_perm, h, y, dy, gu, dgu,
+        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, gu_s, dgu_s, dx_s, dy_s, y_s, total;
     int64_t rp, e_pad;
 };
 
@@ -441,7 +471,7 @@ BwdLayout bwd_layout(const moe_cfg& c)
     L.h = take(rp * I * 2);
     L.y = take(rp * H * 2);
     L.dy = take(rp * H * 2);
-    L.dh = take(rp * I * 2);
+    L.gu = take(rp * 2 * I * 4);
     L.dgu = take(rp * 2 * I * 2);
     L.dx_perm = take(rp * H * 2);
     L.dw_tk = take(A * 4);
@@ -450,7 +480,7 @@ BwdLayout bwd_layout(const moe_cfg& c)
     L.dx_r = take(T * H * 2);
     L.koffT = take(2 * 4);
     L.h_s = take(T * Is * 2);
-    L.dh_s = take(T * Is * 2);
+    L.gu_s = take(T * 2 * Is * 4);
     L.dgu_s = take(T * 2 * Is * 2);
     L.dx_s = take(Is ? T * H * 2 : 0);
     L.dy_s = take(Is ? T * H * 2 : 0);
@@ -513,11 +543,11 @@ int train_intermediates(const moe_cfg& c, const uint16_t* x, const int32_t* ids,
     MOE_TRY(launch_pad_rows(ids, dest_row, offsets, poff, A, E, dest_pad, st));
     MOE_TRY(launch_zero_pad_rows(x_perm, H, offsets, poff, E, st));
     MOE_TRY(launch_gather_rows(c, x, dest_pad, x_perm, st));
-    MOE_TRY(gate_up(x_perm, rp, nullptr, rp, poff, E, 0, w13, H, I, h, status, st));
+    MOE_TRY(gate_up_save(x_perm, rp, poff, E, 0, w13, H, I, h, at<float>(ws, L.gu), status, st));
     MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, at<uint16_t>(ws, L.y), status, st));
     if (Is > 0)
-        MOE_TRY(gate_up(x, T, nullptr, T, nullptr, 1, T, w13s, H, Is, at<uint16_t>(ws, L.h_s),
-                        status, st));
+        MOE_TRY(gate_up_save(x, T, nullptr, 1, T, w13s, H, Is, at<uint16_t>(ws, L.h_s),
+                             at<float>(ws, L.gu_s), status, st));
     return MOE_OK;
 }
 
@@ -541,7 +571,7 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     uint16_t* h = at<uint16_t>(ws, L.h);
     uint16_t* y = at<uint16_t>(ws, L.y);
     uint16_t* dy = at<uint16_t>(ws, L.dy);
-    uint16_t* dh = at<uint16_t>(ws, L.dh);
+    const float* gu = at<float>(ws, L.gu);
     uint16_t* dgu = at<uint16_t>(ws, L.dgu);
     uint16_t* dx_perm = at<uint16_t>(ws, L.dx_perm);
     float* dw_tk = d_topk_w ? d_topk_w : at<float>(ws, L.dw_tk);
@@ -562,10 +592,10 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     uint16_t* dy_s = shared ? at<uint16_t>(ws, L.dy_s) : nullptr;
     MOE_TRY(launch_combine_bwd(c, dout, y, topk_w, dest_pad, mask, dw_tk, dy, dy_s, st));
 
-    // routed experts: dh = dy . W2, dgu (SwiGLU backward on the recomputed gate/up
-    // product), dx rows = dgu . W13; the weights are read MN-major as stored
-    MOE_TRY(gemm_bf16_mn(dy, rp, poff, E, 0, w2, I, H, H, dh, status, st));
-    MOE_TRY(gemm_swiglu_bwd(x_perm, rp, poff, E, 0, w13, H, I, dh, dgu, status, st));
+    // routed experts: dh = dy . W2 in fp32 and, in the same product's epilogue, the SwiGLU
+    // backward dgu from the forward's kept gate/up values; dx rows = dgu . W13; the weights
+    // are read MN-major as stored
+    MOE_TRY(gemm_dswiglu(dy, rp, poff, E, 0, w2, I, H, gu, dgu, status, st));
     MOE_TRY(gemm_bf16_mn(dgu, rp, poff, E, 0, w13, H, 2 * I, 2 * I, dx_perm, status, st));
 
     // router: dlogits, then dx_router = bf16(dlogits) . W_router (K padded to 64: the rows
@@ -577,11 +607,10 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     uint16_t *h_s = nullptr, *dgu_s = nullptr, *dx_s = nullptr;
     if (shared) {
         h_s = at<uint16_t>(ws, L.h_s);
-        uint16_t* dh_s = at<uint16_t>(ws, L.dh_s);
         dgu_s = at<uint16_t>(ws, L.dgu_s);
         dx_s = at<uint16_t>(ws, L.dx_s);
-        MOE_TRY(gemm_bf16_mn(dy_s, T, nullptr, 1, T, w2s, Is, H, H, dh_s, status, st));
-        MOE_TRY(gemm_swiglu_bwd(x, T, nullptr, 1, T, w13s, H, Is, dh_s, dgu_s, status, st));
+        MOE_TRY(gemm_dswiglu(dy_s, T, nullptr, 1, T, w2s, Is, H, at<float>(ws, L.gu_s), dgu_s,
+                             status, st));
         MOE_TRY(gemm_bf16_mn(dgu_s, T, nullptr, 1, T, w13s, H, 2 * Is, 2 * Is, dx_s, status, st));
     }
 

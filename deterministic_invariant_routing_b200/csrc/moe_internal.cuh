@@ -110,7 +110,8 @@ cudaError_t launch_zero_pad_rows(uint16_t* buf, int64_t cols, const int32_t* off
 // tensor-core GEMMs (tcgen05 / TMEM / TMA)
 //   EPI_SWIGLU      out[r, c] = bf16(silu(g) * u) of A . B_g^T (gate and up columns paired)
 //   EPI_BF16        out[r, c] = bf16(A . B_g^T)
-//   EPI_SWIGLU_BWD  the gate/up product recomputed; with dh = aux[r, c] (bf16):
+//   EPI_SWIGLU_SAVE EPI_SWIGLU, also gu[r, c] = g, gu[r, n + c] = u (fp32, as accumulated)
+//   EPI_DSWIGLU     dh = A . B_g^T kept in fp32, g = gu[r, c], u = gu[r, n + c]:
 //                   out[r, c] = bf16(dh * u * silu'(g)), out[r, n + c] = bf16(dh * silu(g))
 //   EPI_WGRAD       grouped over K: out[g][m, c] = fp32(sum over k in [k_offsets[g],
 //                   k_offsets[g+1]) of A[m, k] * B[c, k]) -- an expert's rows contracted
@@ -118,9 +119,10 @@ cudaError_t launch_zero_pad_rows(uint16_t* buf, int64_t cols, const int32_t* off
 enum GemmEpilogue {
     EPI_SWIGLU = 0,
     EPI_BF16 = 1,
-    EPI_SWIGLU_BWD = 2,
     EPI_WGRAD = 3,
-    EPI_F32 = 4
+    EPI_F32 = 4,
+    EPI_SWIGLU_SAVE = 5,
+    EPI_DSWIGLU = 6
 };
 
 struct GemmProblem {
@@ -140,8 +142,8 @@ struct GemmProblem {
     int64_t ldo;             // output row stride in elements
     const float* bias;       // EPI_F32: per-column bias or NULL
     int32_t* status;         // device status words (MOE_ST_PIPE_TIMEOUT) or NULL
-    const uint16_t* aux;     // EPI_SWIGLU_BWD: dh [rows, ld_aux] bf16
-    int64_t ld_aux;
+    float* gu;               // EPI_SWIGLU_SAVE (written) / EPI_DSWIGLU (read): fp32 gate values
+    int64_t ld_gu;           //   at columns [0, n), up values at [n, 2n), row stride ld_gu
     const int32_t* k_offsets;  // EPI_WGRAD: device [groups+1] K ranges (multiples of 64)
     int b_mn;                // B given MN-major, [groups * b_k_rows, n] (K rows of each group,
     int b_k_rows;            //   N contiguous), read without transposing (EPI_WGRAD: [k, n])

@@ -233,6 +233,12 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+// bring the 128-byte line holding p into L2 (no register result, nothing waits for it)
+__device__ __forceinline__ void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared (L1 bypassed), grouped by commit_group
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src)
 {

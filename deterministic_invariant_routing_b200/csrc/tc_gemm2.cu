@@ -61,9 +61,10 @@ struct PairArgs {
     int32_t* status;
     int m_tiles;                 // EPI_WGRAD: row tiles of A (per group)
     const int32_t* k_offsets;    // EPI_WGRAD: [groups+1] K ranges
-    const uint16_t* aux;         // EPI_SWIGLU_BWD: dh
-    int64_t ld_aux;
-    int half_out;                // EPI_SWIGLU_BWD: column of the first up gradient
+    float* gu;                   // EPI_SWIGLU_SAVE / EPI_DSWIGLU: fp32 gate | up values
+    int64_t ld_gu;
+    int half_out;                // EPI_DSWIGLU, EPI_SWIGLU_SAVE: column of the first up
+                                 // value (gradient) in a row
     const float* bias;           // EPI_F32: per-column bias or NULL
     int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
     int skip_tails;              // leave each group's last rows to the 1-SM tail kernel when
@@ -223,7 +224,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     constexpr bool kWgrad = (EPI == EPI_WGRAD);
-    constexpr bool kGateUp = (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD);
+    constexpr bool kGateUp =
+        (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE);
     const int total = kWgrad ? G * args.m_tiles * args.n_tiles : prefix[G] * args.n_tiles;
     auto decode = [&](int t) -> PairTile {
         if (kWgrad) return decode_wgrad_tile(t, args);
@@ -469,6 +471,18 @@ __global__ void __launch_bounds__(kThreads2, 1)
         for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
             const PairTile ti = decode(t);
             const int acc = i & 1;
+            if (EPI == EPI_DSWIGLU) {
+                // this row's gate and up values of the tile into L2 while the MMAs run
+                const int64_t r = ti.row0 + (int64_t)rank * HM + row;
+                if (r < ti.row_end) {
+                    const float* gr = args.gu + r * args.ld_gu + ti.n * NP;
+#pragma unroll
+                    for (int c = 0; c < NP; c += 32) {
+                        prefetch_l2(gr + c);
+                        prefetch_l2(gr + args.half_out + c);
+                    }
+                }
+            }
             int ok = 1;
             if (lane == 0)
                 ok = wait_bounded(tfull_bar(acc), ((uint32_t)i >> 1) & 1u, abort_flag, args.status);
@@ -481,12 +495,23 @@ __global__ void __launch_bounds__(kThreads2, 1)
             const int row_blk = (int)(ti.row0 + (int64_t)rank * HM + q * 32);
             const bool full_blk = (int64_t)row_blk + 31 < ti.row_end;
             uint16_t* out = static_cast<uint16_t*>(args.out);
-            if (EPI == EPI_SWIGLU) {
+            if (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE) {
 #pragma unroll 1
                 for (int c = 0; c < NP / 2; c += 32) {
                     uint32_t g[32], u[32];
                     tmem_ld32(tbase + (uint32_t)c, g);
                     tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
+                    if (EPI == EPI_SWIGLU_SAVE && valid) {
+                        // the fp32 gate and up values, for the backward's SwiGLU derivative
+                        float* gr = args.gu + grow * args.ld_gu + ti.n * (NP / 2) + c;
+                        uint4* dg = reinterpret_cast<uint4*>(gr);
+                        uint4* du = reinterpret_cast<uint4*>(gr + args.half_out);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            dg[v] = make_uint4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
+                            du[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+                        }
+                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
@@ -502,30 +527,36 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     const int col = ti.n * (NP / 2) + c;
                     store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
                 }
-            } else if (EPI == EPI_SWIGLU_BWD) {
-                // dh of this row's 32 intermediate columns, then the SwiGLU derivatives:
-                // silu(g) = g s, s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s))
+            } else if (EPI == EPI_DSWIGLU) {
+                // dh (fp32, this row's 32 intermediate columns) with the kept gate and up
+                // values g, u: dg = dh u silu'(g), du = dh silu(g), where silu(g) = g s,
+                // s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s))
 #pragma unroll 1
-                for (int c = 0; c < NP / 2; c += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld32(tbase + (uint32_t)c, g);
-                    tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
-                    const int col = ti.n * (NP / 2) + c;
-                    uint32_t dhw[16];
+                for (int c = 0; c < NP; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + (uint32_t)c, r);
+                    const int col = ti.n * NP + c;
+                    uint32_t gw[32], uw[32];
                     if (valid) {
-                        const uint4* src =
-                            reinterpret_cast<const uint4*>(args.aux + grow * args.ld_aux + col);
+                        const uint4* sg4 =
+                            reinterpret_cast<const uint4*>(args.gu + grow * args.ld_gu + col);
+                        const uint4* su4 = reinterpret_cast<const uint4*>(
+                            args.gu + grow * args.ld_gu + args.half_out + col);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const uint4 q4 = src[v];
-                            dhw[4 * v] = q4.x;
-                            dhw[4 * v + 1] = q4.y;
-                            dhw[4 * v + 2] = q4.z;
-                            dhw[4 * v + 3] = q4.w;
+                        for (int v = 0; v < 8; ++v) {
+                            const uint4 a4 = sg4[v], b4 = su4[v];
+                            gw[4 * v] = a4.x;
+                            gw[4 * v + 1] = a4.y;
+                            gw[4 * v + 2] = a4.z;
+                            gw[4 * v + 3] = a4.w;
+                            uw[4 * v] = b4.x;
+                            uw[4 * v + 1] = b4.y;
+                            uw[4 * v + 2] = b4.z;
+                            uw[4 * v + 3] = b4.w;
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) dhw[j] = 0u;
+                        for (int j = 0; j < 32; ++j) gw[j] = uw[j] = 0u;
                     }
                     uint32_t pg[16], pu[16];
 #pragma unroll
@@ -533,10 +564,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
                         float dg2[2], du2[2];
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
-                            const float gv = __uint_as_float(g[2 * j + h2]);
-                            const float uv = __uint_as_float(u[2 * j + h2]);
-                            const float dh = __uint_as_float(h2 ? (dhw[j] & 0xffff0000u)
-                                                                : (dhw[j] << 16));
+                            const float gv = __uint_as_float(gw[2 * j + h2]);
+                            const float uv = __uint_as_float(uw[2 * j + h2]);
+                            const float dh = __uint_as_float(r[2 * j + h2]);
                             const float sg = __frcp_rn(1.0f + __expf(-gv));
                             const float dsilu = sg * (1.0f + gv * (1.0f - sg));
                             dg2[h2] = dh * uv * dsilu;
@@ -683,13 +713,14 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (wgrad || EPI == EPI_F32) {
         mo = mb;  // fp32 rows are stored from registers; the store map is not used
     } else {
-        const int out_cols = (EPI == EPI_SWIGLU_BWD) ? 2 * p.n : p.n;
+        const int out_cols = (EPI == EPI_DSWIGLU) ? 2 * p.n : p.n;
         if (!make_store_map(&mo, p.out, rows_total, out_cols, p.ldo))
             return cudaErrorInvalidValue;
     }
     PairArgs a;
     a.k_blocks = p.k / BK;
-    constexpr bool kGateUpL = (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD);
+    constexpr bool kGateUpL =
+        (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE);
     a.n_tiles = kGateUpL ? p.n / (NP / 2) : p.n / NP;
     a.groups = groups;
     a.offsets = p.offsets;
@@ -698,9 +729,10 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.half_rows = kGateUpL ? p.n : 0;
     a.m_tiles = wgrad ? (int)((p.rows + PM - 1) / PM) : 0;
     a.k_offsets = p.k_offsets;
-    a.aux = p.aux;
-    a.ld_aux = p.ld_aux;
-    a.half_out = (EPI == EPI_SWIGLU_BWD) ? p.n : 0;
+    a.half_out =
+        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE) ? p.n : 0;
+    a.gu = p.gu;
+    a.ld_gu = p.ld_gu;
     a.bias = p.bias;
     a.b_k_rows = wgrad ? 0 : p.b_k_rows;
     a.skip_tails = p.skip_tails;
@@ -733,12 +765,22 @@ cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st)
         return launch_pair_variant<EPI_SWIGLU, 256, false>(p, st);
     }
     if (p.gather_rows) return cudaErrorInvalidValue;
+    if (p.epilogue == EPI_SWIGLU_SAVE) {
+        if (p.n % 128 != 0 || p.gu == nullptr || p.ld_gu < 2 * (int64_t)p.n || p.ld_gu % 4 != 0 ||
+            p.b_mn || p.skip_tails)
+            return cudaErrorInvalidValue;
+        return launch_pair_variant<EPI_SWIGLU_SAVE, 256, false>(p, st);
+    }
+    if (p.epilogue == EPI_DSWIGLU) {
+        // dh = A . B with B MN-major (the down weights as stored), N = the intermediate size
+        if (!p.b_mn || p.gu == nullptr || p.ld_gu < 2 * (int64_t)p.n || p.ld_gu % 4 != 0)
+            return cudaErrorInvalidValue;
+        if (p.n % 256 == 0) return launch_pair_variant<EPI_DSWIGLU, 256, false, 1>(p, st);
+        if (p.n % 128 == 0) return launch_pair_variant<EPI_DSWIGLU, 128, false, 1>(p, st);
+        return cudaErrorInvalidValue;
+    }
     if (p.b_mn && p.epilogue != EPI_BF16 && p.epilogue != EPI_F32 && p.epilogue != EPI_WGRAD)
         return cudaErrorInvalidValue;
-    if (p.epilogue == EPI_SWIGLU_BWD) {
-        if (p.n % 128 != 0 || p.aux == nullptr) return cudaErrorInvalidValue;
-        return launch_pair_variant<EPI_SWIGLU_BWD, 256, false>(p, st);
-    }
     if (p.epilogue == EPI_WGRAD) {
         if (p.k_offsets == nullptr || p.rows < 1) return cudaErrorInvalidValue;
         if (p.a_mn != p.b_mn) return cudaErrorInvalidValue;
