@@ -25,10 +25,14 @@
 // (the leader posts the byte count of both CTAs); the leader's single MMA thread waits on
 // full[s], issues the pair MMAs and commits to empty[s] of both CTAs (multicast commit).
 // Accumulators: the commit of the last k-block arrives on tfull[a] of both CTAs; each
-// CTA's epilogue drains its own TMEM rows and arrives on the leader's tempty[a] (256
-// arrivals). Every wait is bounded and a give-up is recorded in MOE_ST_PIPE_TIMEOUT.
+// CTA's epilogue drains its own TMEM rows and arrives on the leader's tempty[a] (one
+// arrival per epilogue thread of both CTAs). Every wait is bounded and a give-up is
+// recorded in MOE_ST_PIPE_TIMEOUT.
 //
 // Output: each epilogue warp owns 32 accumulator rows and writes them 32 columns at a time.
+// Epilogues that move more global bytes per tile than the main loop hides (the fp32
+// outputs and the SwiGLU backward's gate/up reads) run two warps per 32 rows, each taking
+// every other 32-column chunk.
 // A block whose 32 rows all lie inside the group goes through a 2 KiB shared-memory tile
 // (64-byte swizzle, two per warp, alternating) and one TMA store; the partial block at a
 // group's end is stored row by row from registers, so no padding row reaches global memory.
@@ -41,7 +45,6 @@ namespace {
 
 constexpr int PM = 256;                     // rows per pair tile
 constexpr int HM = 128;                     // rows per CTA = TMEM lanes
-constexpr int kThreads2 = 192;
 constexpr uint32_t kA2Bytes = HM * BK * 2;  // 16 KiB per stage
 constexpr uint16_t kPairMask = 0x3;
 
@@ -74,13 +77,23 @@ struct PairArgs {
 template <int EPI, int NP>
 struct Cfg2 {
     static_assert(NP == 128 || NP == 256, "pair N");
+    // epilogue warps: two per TMEM lane quarter (each taking every other 32-column chunk)
+    // where the epilogue moves more global bytes than the main loop hides with one
+    static constexpr int kEpiWarps =
+        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD) ? 8 : 4;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    // bf16 outputs go through two 32 x 32 store tiles per epilogue warp; fp32 rows are
+    // written from registers
+    static constexpr uint32_t kEpiBytes =
+        (EPI == EPI_WGRAD || EPI == EPI_F32) ? 0u : (uint32_t)kEpiWarps * 2u * 2048u;
     static constexpr uint32_t kBBytes = (uint32_t)(NP / 2) * BK * 2;  // this CTA's half of B
     static constexpr uint32_t kStageBytes = kA2Bytes + kBBytes;
-    static constexpr int kStages0 = kSmemBudget / (int)kStageBytes;
+    // the operand ring gives up what the store tiles take beyond four warps' worth
+    static constexpr int kRing = kSmemBudget - (kEpiBytes > 16384u ? (int)kEpiBytes - 16384 : 0);
+    static constexpr int kStages0 = kRing / (int)kStageBytes;
     static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
     static constexpr uint32_t kTmemCols = 2 * NP;
     static constexpr int kBars = 2 * kStages + 5;
-    static constexpr uint32_t kEpiBytes = 4 * 2 * 2048;  // 4 warps x 2 tiles of 32 x 32 bf16
     static size_t smem_bytes(int groups)
     {
         return 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kBars * 8 + 16 +
@@ -136,7 +149,7 @@ __device__ __forceinline__ PairTile decode_wgrad_tile(int t, const PairArgs& a)
 // MN: operand majorness fixed at compile time -- 0 both K-major, 1 B MN-major, 2 A and B
 // MN-major (the weight-gradient products)
 template <int EPI, int NP, bool GATHER, int MN>
-__global__ void __launch_bounds__(kThreads2, 1)
+__global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmO, PairArgs args)
@@ -180,7 +193,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 2 * 4 * 32);
+            mbar_init(tempty_bar(a), 2 * C::kEpiWarps * 32);
         }
         mbar_init(drain_bar, 1);
         misc[1] = 0;
@@ -430,11 +443,14 @@ __global__ void __launch_bounds__(kThreads2, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue
-        const int q = warp & 3;
+        const int q = warp & 3;  // TMEM lanes 32 q .. 32 q + 31 (a warp's lane quarter is warp % 4)
         const int row = q * 32 + lane;
+        constexpr bool kTwo = C::kEpiWarps == 8;
+        constexpr int cstep = kTwo ? 64 : 32;          // chunk stride of this warp's columns
+        const int c0 = kTwo ? 32 * ((warp - 2) >> 2) : 0;  // and its first chunk
         const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
         const uint32_t tempty_leader1 = mapa_shared(tempty_bar(1), 0);
-        const uint32_t ebuf = sE0 + (uint32_t)q * 4096u;
+        const uint32_t ebuf = sE0 + (uint32_t)(kTwo ? warp - 2 : q) * 4096u;
         uint32_t eb = 0;  // which of the warp's two store tiles is next
         // this lane's row of a store tile: 64 bytes, 16-byte chunks at the swizzled place
         const uint32_t erow = (uint32_t)lane * 64u, eswz = ((uint32_t)lane >> 1) & 3u;
@@ -477,7 +493,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 if (r < ti.row_end) {
                     const float* gr = args.gu + r * args.ld_gu + ti.n * NP;
 #pragma unroll
-                    for (int c = 0; c < NP; c += 32) {
+                    for (int c = c0; c < NP; c += cstep) {
                         prefetch_l2(gr + c);
                         prefetch_l2(gr + args.half_out + c);
                     }
@@ -497,7 +513,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
             uint16_t* out = static_cast<uint16_t*>(args.out);
             if (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE) {
 #pragma unroll 1
-                for (int c = 0; c < NP / 2; c += 32) {
+                for (int c = c0; c < NP / 2; c += cstep) {
                     uint32_t g[32], u[32];
                     tmem_ld32(tbase + (uint32_t)c, g);
                     tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
@@ -532,7 +548,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 // values g, u: dg = dh u silu'(g), du = dh silu(g), where silu(g) = g s,
                 // s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s))
 #pragma unroll 1
-                for (int c = 0; c < NP; c += 32) {
+                for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
                     tmem_ld32(tbase + (uint32_t)c, r);
                     const int col = ti.n * NP + c;
@@ -583,7 +599,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 // fp32 rows plus the column bias (the router's logits)
                 float* o = static_cast<float*>(args.out);
 #pragma unroll 1
-                for (int c = 0; c < NP; c += 32) {
+                for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
                     tmem_ld32(tbase + (uint32_t)c, r);
                     const int col = ti.n * NP + c;
@@ -603,7 +619,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 // fp32 weight gradient rows of group g; a group with no rows gives zeros
                 float* o = static_cast<float*>(args.out);
 #pragma unroll 1
-                for (int c = 0; c < NP; c += 32) {
+                for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
                     if (ti.kbs > 0) {
                         tmem_ld32(tbase + (uint32_t)c, r);
@@ -621,7 +637,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < NP; c += 32) {
+                for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
                     tmem_ld32(tbase + (uint32_t)c, r);
                     uint32_t pk[16];
@@ -654,6 +670,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     auto kernel = tc_gemm_pair_kernel<EPI, NP, GATHER, MN>;
     const int groups = (p.offsets || EPI == EPI_WGRAD) ? p.groups : 1;
     const size_t smem = C::smem_bytes(groups);
+    if (smem > 232448) return cudaErrorInvalidValue;  // more groups than shared memory holds
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -668,7 +685,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(kThreads2, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
