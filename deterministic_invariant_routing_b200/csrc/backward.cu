@@ -261,6 +261,35 @@ __global__ void __launch_bounds__(1024) padded_offsets_kernel(const int32_t* __r
     if (g == 0) poff[0] = 0;
 }
 
+// K ranges of a product over `rows` rows split into chunks of `chunk` rows (a multiple of
+// 64): koff[s] = min(s * chunk, rows rounded up to 64), s = 0..S
+__global__ void split_offsets_kernel(int rows, int chunk, int S, int32_t* __restrict__ koff)
+{
+    pdl_wait();
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    const int end = (rows + 63) / 64 * 64;
+    if (s <= S) koff[s] = (int)((int64_t)s * chunk < end ? (int64_t)s * chunk : end);
+}
+
+// out[i] = part[0][i] + part[1][i] + ... + part[S-1][i], fp32 adds in chunk order
+__global__ void __launch_bounds__(256) sum_parts_kernel(const float4* __restrict__ part, int S,
+                                                        int64_t n4, float4* __restrict__ out)
+{
+    pdl_wait();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = part[i];
+        for (int s = 1; s < S; ++s) {
+            const float4 b = part[(int64_t)s * n4 + i];
+            a.x = __fadd_rn(a.x, b.x);
+            a.y = __fadd_rn(a.y, b.y);
+            a.z = __fadd_rn(a.z, b.z);
+            a.w = __fadd_rn(a.w, b.w);
+        }
+        out[i] = a;
+    }
+}
+
 __global__ void pad_rows_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ dest,
                                 const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
                                 int64_t A, int E, int32_t* __restrict__ dest_pad)
@@ -350,6 +379,25 @@ cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* 
 {
     if (G < 1 || G > 1024) return cudaErrorInvalidValue;
     return launch_pdl(padded_offsets_kernel, dim3(1), dim3(1024), 0, st, off, G, rows, poff);
+}
+
+cudaError_t launch_split_offsets(int rows, int chunk, int S, int32_t* koff, cudaStream_t st)
+{
+    if (S < 1 || chunk < 64 || chunk % 64 != 0) return cudaErrorInvalidValue;
+    return launch_pdl(split_offsets_kernel, dim3((unsigned)((S + 1 + 255) / 256)), dim3(256), 0,
+                      st, rows, chunk, S, koff);
+}
+
+cudaError_t launch_sum_parts(const float* part, int S, int64_t n, float* out, cudaStream_t st)
+{
+    if (S < 1 || n % 4 != 0) return cudaErrorInvalidValue;
+    const int64_t n4 = n / 4;
+    if (n4 == 0) return cudaSuccess;
+    int64_t blocks = (n4 + 255) / 256;
+    const int64_t cap = resident_blocks((const void*)sum_parts_kernel, 256, 0);
+    if (blocks > cap) blocks = cap;
+    return launch_pdl(sum_parts_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                      reinterpret_cast<const float4*>(part), S, n4, reinterpret_cast<float4*>(out));
 }
 
 cudaError_t launch_pad_rows(const int32_t* ids, const int32_t* dest_row, const int32_t* off,

@@ -444,9 +444,29 @@ size_t pad64(size_t v) { return (v + 63) / 64 * 64; }
 // form whole 64-row K blocks of the weight-gradient products.
 struct BwdLayout {
     size_t offsets, perm_token, dest_row, dest_pad, poff, perm_ws, x_perm, h, y, dy, gu, dgu,
-        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, h_s, gu_s, dgu_s, dx_s, dy_s, y_s, total;
+        dx_perm, dw_tk, dl, dl_bf, dx_r, koffT, koffS, wr_part, h_s, gu_s, dgu_s, dx_s, dy_s,
+        y_s, total;
     int64_t rp, e_pad;
 };
+
+// K splits of the router's weight-gradient product (E x H outputs, K = T tokens): its output
+// makes only ceil(E / 256) * H / 256 tiles, too few for the GPU's CTA pairs, so the tokens
+// are cut into S chunks of a multiple of 64 (S partial products, then one in-order sum);
+// enough chunks for two tiles per pair of a 148-SM B200. A function of (E, H, T) only, so
+// the bits do not depend on the device.
+int router_wgrad_splits(int E, int H, int T, int* chunk)
+{
+    constexpr int64_t kPairs = 74;
+    const int64_t tiles = ((E + 255) / 256) * (H % 256 == 0 ? H / 256 : H / 128);
+    int64_t S = 1;
+    if (tiles > 0 && tiles < kPairs) S = (2 * kPairs + tiles - 1) / tiles;
+    int64_t ch = (((int64_t)T + S - 1) / S + 63) / 64 * 64;
+    if (ch < 64) ch = 64;
+    S = ((int64_t)T + ch - 1) / ch;
+    if (S < 1) S = 1;
+    *chunk = (int)ch;
+    return (int)S;
+}
 
 BwdLayout bwd_layout(const moe_cfg& c)
 {
@@ -479,6 +499,10 @@ BwdLayout bwd_layout(const moe_cfg& c)
     L.dl_bf = take(T * ep * 2);
     L.dx_r = take(T * H * 2);
     L.koffT = take(2 * 4);
+    int chunk = 0;
+    const size_t S = (size_t)router_wgrad_splits(c.E, c.H, c.T, &chunk);
+    L.koffS = take((S + 1) * 4);
+    L.wr_part = take(S > 1 ? S * c.E * H * 4 : 0);
     L.h_s = take(T * Is * 2);
     L.gu_s = take(T * 2 * Is * 4);
     L.dgu_s = take(T * 2 * Is * 2);
@@ -623,7 +647,18 @@ int backward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* wr, const
     MOE_TRY(gemm_wgrad_mn(dy, H, H, h, I, rp, poff, E, dw2, status, st));
     MOE_TRY(gemm_wgrad_mn(dgu, 2 * I, 2 * I, x_perm, H, rp, poff, E, dw13, status, st));
     MOE_TRY(launch_padded_offsets(nullptr, 1, T, koffT, st));
-    MOE_TRY(gemm_wgrad_mn(dl_bf, ep, E, x, H, T, koffT, 1, dwr, status, st));
+    int chunk = 0;
+    const int S = router_wgrad_splits(E, H, T, &chunk);
+    if (S > 1) {
+        // the router's product split over K (chunks of tokens), partials summed in order
+        int32_t* koffS = at<int32_t>(ws, L.koffS);
+        float* part = at<float>(ws, L.wr_part);
+        MOE_TRY(launch_split_offsets(T, chunk, S, koffS, st));
+        MOE_TRY(gemm_wgrad_mn(dl_bf, ep, E, x, H, T, koffS, S, part, status, st));
+        MOE_TRY(launch_sum_parts(part, S, (int64_t)E * H, dwr, st));
+    } else {
+        MOE_TRY(gemm_wgrad_mn(dl_bf, ep, E, x, H, T, koffT, 1, dwr, status, st));
+    }
     if (shared) {
         MOE_TRY(gemm_wgrad_mn(dy_s, H, H, h_s, Is, T, koffT, 1, dw2s, status, st));
         MOE_TRY(gemm_wgrad_mn(dgu_s, 2 * Is, 2 * Is, x, H, T, koffT, 1, dw13s, status, st));

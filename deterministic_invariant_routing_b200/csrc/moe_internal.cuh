@@ -98,6 +98,10 @@ cudaError_t launch_unpermute(const moe_cfg& c, const uint16_t* rows, const int32
                              uint16_t* dx, cudaStream_t st);
 cudaError_t launch_padded_offsets(const int32_t* off, int G, int rows, int32_t* poff,
                                   cudaStream_t st);
+// split-K of a K-grouped product: koff[s] = min(s * chunk, rows rounded up to 64), s = 0..S
+cudaError_t launch_split_offsets(int rows, int chunk, int S, int32_t* koff, cudaStream_t st);
+// out[i] = sum over s = 0..S-1 in order of part[s * n + i] (n a multiple of 4)
+cudaError_t launch_sum_parts(const float* part, int S, int64_t n, float* out, cudaStream_t st);
 // dest_row (dispatch rows) -> rows of the layout whose expert ranges start at poff (each
 // padded to 64 rows): r' = poff[e] + (r - off[e]), e = ids[a]; -1 stays -1
 cudaError_t launch_pad_rows(const int32_t* ids, const int32_t* dest_row, const int32_t* off,

@@ -82,10 +82,10 @@ struct Cfg2 {
     static constexpr int kEpiWarps =
         (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD) ? 8 : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
-    // bf16 outputs go through two 32 x 32 store tiles per epilogue warp; fp32 rows are
-    // written from registers
+    // outputs go through two 2 KiB store tiles per epilogue warp (32 rows of 32 bf16 or 16
+    // fp32 values); the router's fp32 logits are written from registers
     static constexpr uint32_t kEpiBytes =
-        (EPI == EPI_WGRAD || EPI == EPI_F32) ? 0u : (uint32_t)kEpiWarps * 2u * 2048u;
+        (EPI == EPI_F32) ? 0u : (uint32_t)kEpiWarps * 2u * 2048u;
     static constexpr uint32_t kBBytes = (uint32_t)(NP / 2) * BK * 2;  // this CTA's half of B
     static constexpr uint32_t kStageBytes = kA2Bytes + kBBytes;
     // the operand ring gives up what the store tiles take beyond four warps' worth
@@ -152,7 +152,8 @@ template <int EPI, int NP, bool GATHER, int MN>
 __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmO, PairArgs args)
+                        const __grid_constant__ CUtensorMap tmO,
+                        const __grid_constant__ CUtensorMap tmG, PairArgs args)
 {
     using C = Cfg2<EPI, NP>;
     constexpr int S = C::kStages;
@@ -457,7 +458,8 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
         // 32 x 32 block of rows [row_blk, +32), columns [col, +32): through shared memory
         // and TMA when the whole block is inside the group, else the valid rows directly
         auto store_block = [&](const uint32_t (&pk)[16], bool full_blk, bool valid,
-                               int row_blk, int col, uint16_t* dst_row) {
+                               int row_blk, int col, uint16_t* dst_row,
+                               const CUtensorMap* map) {
             if (full_blk) {
                 const uint32_t b = ebuf + eb * 2048u;
                 if (lane == 0) bulk_wait_read<1>();  // the tile stored two blocks ago is read
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmO, b, col, row_blk);
+                    tma_store_2d(map, b, col, row_blk);
                     bulk_commit();
                 }
                 eb ^= 1u;
@@ -517,15 +519,20 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                     uint32_t g[32], u[32];
                     tmem_ld32(tbase + (uint32_t)c, g);
                     tmem_ld32(tbase + (uint32_t)(NP / 2 + c), u);
-                    if (EPI == EPI_SWIGLU_SAVE && valid) {
-                        // the fp32 gate and up values, for the backward's SwiGLU derivative
-                        float* gr = args.gu + grow * args.ld_gu + ti.n * (NP / 2) + c;
-                        uint4* dg = reinterpret_cast<uint4*>(gr);
-                        uint4* du = reinterpret_cast<uint4*>(gr + args.half_out);
+                    if (EPI == EPI_SWIGLU_SAVE) {
+                        // the fp32 gate and up values, for the backward's SwiGLU derivative:
+                        // four 16-column store tiles
+                        const int gcol = ti.n * (NP / 2) + c;
+                        float* gr = args.gu + grow * args.ld_gu + gcol;
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            dg[v] = make_uint4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
-                            du[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+                        for (int part = 0; part < 4; ++part) {
+                            const uint32_t* src = (part < 2 ? g : u) + 16 * (part & 1);
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pk[j] = src[j];
+                            const int off = (part < 2 ? 0 : args.half_out) + 16 * (part & 1);
+                            store_block(pk, full_blk, valid, row_blk, gcol + off,
+                                        reinterpret_cast<uint16_t*>(gr + off), &tmG);
                         }
                     }
                     uint32_t pk[16];
@@ -541,7 +548,8 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                         pk[j] = bf16x2_rne(hv[0], hv[1]);
                     }
                     const int col = ti.n * (NP / 2) + c;
-                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
+                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col,
+                                &tmO);
                 }
             } else if (EPI == EPI_DSWIGLU) {
                 // dh (fp32, this row's 32 intermediate columns) with the kept gate and up
@@ -591,9 +599,11 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                         pg[j] = bf16x2_rne(dg2[0], dg2[1]);
                         pu[j] = bf16x2_rne(du2[0], du2[1]);
                     }
-                    store_block(pg, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
+                    store_block(pg, full_blk, valid, row_blk, col, out + grow * args.ldo + col,
+                                &tmO);
                     const int ucol = args.half_out + col;
-                    store_block(pu, full_blk, valid, row_blk, ucol, out + grow * args.ldo + ucol);
+                    store_block(pu, full_blk, valid, row_blk, ucol, out + grow * args.ldo + ucol,
+                                &tmO);
                 }
             } else if (EPI == EPI_F32) {
                 // fp32 rows plus the column bias (the router's logits)
@@ -616,8 +626,10 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                     }
                 }
             } else if (EPI == EPI_WGRAD) {
-                // fp32 weight gradient rows of group g; a group with no rows gives zeros
+                // fp32 weight gradient rows of group g (rows g * rows + m of the output), 16
+                // columns per store tile; a group with no rows gives zeros
                 float* o = static_cast<float*>(args.out);
+                const int orow_blk = ti.g * args.rows + row_blk;
 #pragma unroll 1
                 for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
@@ -627,13 +639,18 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) r[j] = 0u;
                     }
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            o + ((int64_t)ti.g * args.rows + grow) * args.ldo + ti.n * NP + c);
+                    uint32_t lo[16], hi[16];
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                    for (int j = 0; j < 16; ++j) {
+                        lo[j] = r[j];
+                        hi[j] = r[16 + j];
                     }
+                    const int col = ti.n * NP + c;
+                    float* drow = o + ((int64_t)ti.g * args.rows + grow) * args.ldo + col;
+                    store_block(lo, full_blk, valid, orow_blk, col,
+                                reinterpret_cast<uint16_t*>(drow), &tmO);
+                    store_block(hi, full_blk, valid, orow_blk, col + 16,
+                                reinterpret_cast<uint16_t*>(drow + 16), &tmO);
                 }
             } else {
 #pragma unroll 1
@@ -645,7 +662,8 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                     for (int j = 0; j < 16; ++j)
                         pk[j] = bf16x2_rne(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
                     const int col = ti.n * NP + c;
-                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col);
+                    store_block(pk, full_blk, valid, row_blk, col, out + grow * args.ldo + col,
+                                &tmO);
                 }
             }
             tc_fence_before();
@@ -709,7 +727,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
         max_smem[dev] = smem;
     }
     const int64_t rows_total = p.offsets ? p.a_rows_total : p.rows;
-    CUtensorMap ma, mb, mo;
+    CUtensorMap ma, mb, mo, mg;
     const bool wgrad = (EPI == EPI_WGRAD);
     if (p.a_mn) {
         // [k, a_rows] with the features contiguous: boxes of 64 features x 64 K rows
@@ -727,7 +745,11 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
                          NP / 2)) {
         return cudaErrorInvalidValue;
     }
-    if (wgrad || EPI == EPI_F32) {
+    if (wgrad) {
+        // [groups * rows, n] fp32 in 32 x 16 store tiles
+        if (!make_store_map_f32(&mo, p.out, (int64_t)groups * p.rows, p.n, p.ldo))
+            return cudaErrorInvalidValue;
+    } else if (EPI == EPI_F32) {
         mo = mb;  // fp32 rows are stored from registers; the store map is not used
     } else {
         const int out_cols = (EPI == EPI_DSWIGLU) ? 2 * p.n : p.n;
@@ -765,7 +787,14 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (max_tiles < clusters) clusters = max_tiles;
     if (clusters < 1) clusters = 1;
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mo, a);
+    if (EPI == EPI_SWIGLU_SAVE) {
+        // the kept gate | up values: fp32 [rows, ld_gu] in 32 x 16 store tiles
+        if (!make_store_map_f32(&mg, p.gu, rows_total, 2 * (int64_t)p.n, p.ld_gu))
+            return cudaErrorInvalidValue;
+    } else {
+        mg = mo;  // not used
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mo, mg, a);
 }
 
 }  // namespace
