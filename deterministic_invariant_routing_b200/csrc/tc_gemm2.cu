@@ -86,17 +86,21 @@ struct Cfg2 {
     // fp32 values); the router's fp32 logits are written from registers
     static constexpr uint32_t kEpiBytes =
         (EPI == EPI_F32) ? 0u : (uint32_t)kEpiWarps * 2u * 2048u;
+    // EPI_DSWIGLU: per epilogue warp a 4 KiB tile of the kept gate and up values (32 rows x
+    // 16 fp32 each) loaded by TMA, and its barrier
+    static constexpr uint32_t kGuBytes = (EPI == EPI_DSWIGLU) ? (uint32_t)kEpiWarps * 4096u : 0u;
     static constexpr uint32_t kBBytes = (uint32_t)(NP / 2) * BK * 2;  // this CTA's half of B
     static constexpr uint32_t kStageBytes = kA2Bytes + kBBytes;
-    // the operand ring gives up what the store tiles take beyond four warps' worth
-    static constexpr int kRing = kSmemBudget - (kEpiBytes > 16384u ? (int)kEpiBytes - 16384 : 0);
+    // the operand ring gives up what the epilogue tiles take beyond four warps' store tiles
+    static constexpr int kEpiAll = (int)(kEpiBytes + kGuBytes);
+    static constexpr int kRing = kSmemBudget - (kEpiAll > 16384 ? kEpiAll - 16384 : 0);
     static constexpr int kStages0 = kRing / (int)kStageBytes;
     static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
     static constexpr uint32_t kTmemCols = 2 * NP;
-    static constexpr int kBars = 2 * kStages + 5;
+    static constexpr int kBars = 2 * kStages + 5 + (EPI == EPI_DSWIGLU ? kEpiWarps : 0);
     static size_t smem_bytes(int groups)
     {
-        return 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kBars * 8 + 16 +
+        return 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kGuBytes + kBars * 8 + 16 +
                (size_t)2 * (groups + 1) * sizeof(int32_t) + HM * sizeof(int32_t);
     }
 };
@@ -168,13 +172,16 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     const uint32_t sA0 = smem_u32(base);
     const uint32_t sB0 = sA0 + S * kA2Bytes;
     const uint32_t sE0 = sA0 + S * C::kStageBytes;  // epilogue store tiles
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * C::kStageBytes + C::kEpiBytes);
+    const uint32_t sG0 = sE0 + C::kEpiBytes;          // EPI_DSWIGLU: gate/up tiles
+    uint64_t* bars =
+        reinterpret_cast<uint64_t*>(base + S * C::kStageBytes + C::kEpiBytes + C::kGuBytes);
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(S + s); };
     auto tfull_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (uint32_t)(2 * S + 4);
+    auto gu_bar = [&](int w) { return bar0 + 8u * (uint32_t)(2 * S + 5 + w); };
     uint32_t* misc = reinterpret_cast<uint32_t*>(bars + C::kBars);  // [0] tmem, [1] abort
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     int32_t* prefix = reinterpret_cast<int32_t*>(misc + 4);
@@ -197,6 +204,8 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
             mbar_init(tempty_bar(a), 2 * C::kEpiWarps * 32);
         }
         mbar_init(drain_bar, 1);
+        if (EPI == EPI_DSWIGLU)
+            for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(gu_bar(w), 1);
         misc[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -485,12 +494,24 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                     dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
         };
+        // EPI_DSWIGLU: this warp's gate/up tile (g at +0, u at +2 KiB; 64-byte rows, 64-byte
+        // swizzle) and its barrier; one 16-column load is in flight at a time
+        const uint32_t gbuf = sG0 + (uint32_t)(warp - 2) * 4096u;
+        const uint32_t gbar = gu_bar(warp - 2);
+        uint32_t gphase = 0;
+        bool gu_pending = false, gu_ok = true;
+        auto gu_issue = [&](int row_blk_, int col_) {
+            mbar_expect_tx(gbar, 4096u);
+            tma_load_2d(gbuf, &tmG, col_, row_blk_, gbar);
+            tma_load_2d(gbuf + 2048u, &tmG, args.half_out + col_, row_blk_, gbar);
+        };
         int i = 0;
         for (int t = cluster; t < total && !*abort_flag; t += nclusters, ++i) {
             const PairTile ti = decode(t);
             const int acc = i & 1;
             if (EPI == EPI_DSWIGLU) {
-                // this row's gate and up values of the tile into L2 while the MMAs run
+                // this row's gate and up values of the tile into L2 while the MMAs run, and
+                // the warp's first 16-column tile of them into shared memory
                 const int64_t r = ti.row0 + (int64_t)rank * HM + row;
                 if (r < ti.row_end) {
                     const float* gr = args.gu + r * args.ld_gu + ti.n * NP;
@@ -499,6 +520,11 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                         prefetch_l2(gr + c);
                         prefetch_l2(gr + args.half_out + c);
                     }
+                }
+                if (gu_ok) {
+                    if (lane == 0)
+                        gu_issue((int)(ti.row0 + (int64_t)rank * HM + q * 32), ti.n * NP + c0);
+                    gu_pending = true;
                 }
             }
             int ok = 1;
@@ -554,50 +580,75 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
             } else if (EPI == EPI_DSWIGLU) {
                 // dh (fp32, this row's 32 intermediate columns) with the kept gate and up
                 // values g, u: dg = dh u silu'(g), du = dh silu(g), where silu(g) = g s,
-                // s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s))
+                // s = 1 / (1 + e^-g), silu'(g) = s (1 + g (1 - s)). g and u come 16 columns
+                // at a time through the warp's shared-memory tile; the next 16 are loaded
+                // while these are computed.
+                const uint32_t grow_s = gbuf + (uint32_t)lane * 64u;
+                const uint32_t gswz = ((uint32_t)lane >> 1) & 3u;
+                const int row_blk_g = (int)(ti.row0 + (int64_t)rank * HM + q * 32);
 #pragma unroll 1
                 for (int c = c0; c < NP; c += cstep) {
                     uint32_t r[32];
                     tmem_ld32(tbase + (uint32_t)c, r);
                     const int col = ti.n * NP + c;
-                    uint32_t gw[32], uw[32];
-                    if (valid) {
-                        const uint4* sg4 =
-                            reinterpret_cast<const uint4*>(args.gu + grow * args.ld_gu + col);
-                        const uint4* su4 = reinterpret_cast<const uint4*>(
-                            args.gu + grow * args.ld_gu + args.half_out + col);
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            const uint4 a4 = sg4[v], b4 = su4[v];
-                            gw[4 * v] = a4.x;
-                            gw[4 * v + 1] = a4.y;
-                            gw[4 * v + 2] = a4.z;
-                            gw[4 * v + 3] = a4.w;
-                            uw[4 * v] = b4.x;
-                            uw[4 * v + 1] = b4.y;
-                            uw[4 * v + 2] = b4.z;
-                            uw[4 * v + 3] = b4.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) gw[j] = uw[j] = 0u;
-                    }
                     uint32_t pg[16], pu[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float dg2[2], du2[2];
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const float gv = __uint_as_float(gw[2 * j + h2]);
-                            const float uv = __uint_as_float(uw[2 * j + h2]);
-                            const float dh = __uint_as_float(r[2 * j + h2]);
-                            const float sg = __frcp_rn(1.0f + __expf(-gv));
-                            const float dsilu = sg * (1.0f + gv * (1.0f - sg));
-                            dg2[h2] = dh * uv * dsilu;
-                            du2[h2] = dh * (gv * sg);
+                    for (int h = 0; h < 2; ++h) {
+                        // every lane waits: the barrier's completion makes the copy's
+                        // bytes visible to the waiting thread
+                        if (gu_pending) {
+                            if (wait_bounded(gbar, gphase, abort_flag, args.status)) {
+                                gphase ^= 1u;
+                                gu_pending = false;
+                            } else {
+                                gu_ok = false;  // still in flight: drained before exit
+                            }
                         }
-                        pg[j] = bf16x2_rne(dg2[0], dg2[1]);
-                        pu[j] = bf16x2_rne(du2[0], du2[1]);
+                        uint32_t gw[16], uw[16];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const uint32_t off = (((uint32_t)v) ^ gswz) << 4;
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(gw[4 * v]), "=r"(gw[4 * v + 1]),
+                                           "=r"(gw[4 * v + 2]), "=r"(gw[4 * v + 3])
+                                         : "r"(grow_s + off)
+                                         : "memory");
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(uw[4 * v]), "=r"(uw[4 * v + 1]),
+                                           "=r"(uw[4 * v + 2]), "=r"(uw[4 * v + 3])
+                                         : "r"(grow_s + 2048u + off)
+                                         : "memory");
+                        }
+                        // the tile is read -- each lane's loads have returned (the values
+                        // are used) and are ordered before the copy engine's next writes --
+                        // so the next 16 columns may land in it
+                        uint32_t used = 0;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) used |= gw[j] ^ uw[j];
+                        asm volatile("" ::"r"(used));
+                        fence_async_smem();
+                        __syncwarp();
+                        const int ncol = h == 0 ? col + 16 : col + cstep;
+                        if (gu_ok && (h == 0 || c + cstep < NP)) {
+                            if (lane == 0) gu_issue(row_blk_g, ncol);
+                            gu_pending = true;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float dg2[2], du2[2];
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const float gv = __uint_as_float(gw[2 * j + h2]);
+                                const float uv = __uint_as_float(uw[2 * j + h2]);
+                                const float dh = __uint_as_float(r[16 * h + 2 * j + h2]);
+                                const float sg = __frcp_rn(1.0f + __expf(-gv));
+                                const float dsilu = sg * (1.0f + gv * (1.0f - sg));
+                                dg2[h2] = dh * uv * dsilu;
+                                du2[h2] = dh * (gv * sg);
+                            }
+                            pg[8 * h + j] = bf16x2_rne(dg2[0], dg2[1]);
+                            pu[8 * h + j] = bf16x2_rne(du2[0], du2[1]);
+                        }
                     }
                     store_block(pg, full_blk, valid, row_blk, col, out + grow * args.ldo + col,
                                 &tmO);
@@ -669,6 +720,8 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
             tc_fence_before();
             mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
         }
+        if (EPI == EPI_DSWIGLU && gu_pending)
+            wait_bounded(gbar, gphase, abort_flag, args.status, false);  // no load in flight
         if (lane == 0) bulk_wait_all();  // the TMA stores have written global memory
     }
 
@@ -787,8 +840,8 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     if (max_tiles < clusters) clusters = max_tiles;
     if (clusters < 1) clusters = 1;
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-    if (EPI == EPI_SWIGLU_SAVE) {
-        // the kept gate | up values: fp32 [rows, ld_gu] in 32 x 16 store tiles
+    if (EPI == EPI_SWIGLU_SAVE || EPI == EPI_DSWIGLU) {
+        // the kept gate | up values: fp32 [rows, ld_gu] in 32 x 16 tiles (stored / loaded)
         if (!make_store_map_f32(&mg, p.gu, rows_total, 2 * (int64_t)p.n, p.ld_gu))
             return cudaErrorInvalidValue;
     } else {
