@@ -51,6 +51,14 @@ def parse():
                         "the backward")
     p.add_argument("--extras-reps", type=int, default=20,
                    help="timed repetitions of each extra call")
+    p.add_argument("--split-steps", type=int, default=200,
+                   help="steps of the separate pass that records the per-stage events")
+    p.add_argument("--sweep", action="store_true",
+                   help="instead of the bench line: tokens/s of the layer forward at each batch "
+                        "size of the invariance sweep (one JSON object)")
+    p.add_argument("--oracle-sweep", action="store_true",
+                   help="instead of the bench line: the oracle's tokens/s on the host cores for "
+                        "each workload (one JSON object)")
     return p.parse_args()
 
 
@@ -339,10 +347,92 @@ def time_extras(cfg, layer, x, b, moe, torch, hbm_gbs, tflops, reps=20):
     }
 
 
+BATCH_SWEEP = [1, 2, 3, 7, 16, 64, 255, 256, 1000, 2047, 2048, 2049, 4096, 8192, 16384]
+
+
+def run_sweep(a):
+    """Tokens/s of the layer forward at each batch size of the invariance sweep (the same
+    batch sizes as the bit-equality tests), inputs resident in HBM. Between timed calls a
+    256 MiB buffer is written so that small batches do not find their experts' weights in
+    L2 from the previous call. One JSON object on stdout."""
+    import torch
+
+    from deterministic_invariant_routing_b200 import moe, synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = synthetic.shape(a.workload, T=max(BATCH_SWEEP))
+    weights = synthetic.make_weights(s, device=dev)
+    x_all = synthetic.make_tokens(s, s.T, seed=s.seed + 5, device=dev)
+    cfg = moe.Config.of(s)
+    layer = moe.MoELayer(cfg, weights)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for B in BATCH_SWEEP:
+        x = x_all[:B].contiguous()
+        for _ in range(3):
+            layer(x, check=False)
+        reps = 50 if B < 4096 else 20
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            layer(x, check=False)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        moe.check_status(layer.status)
+        ms = statistics.median(ts)
+        rows.append({"B": B, "ms": ms, "tokens_per_s": B / (ms * 1e-3)})
+    print(json.dumps({"sweep": f"{s.name} layer forward by batch size", "l2": "256 MiB "
+                      "written between calls", "timing": "median of CUDA-event-timed calls",
+                      "rows": rows}), flush=True)
+
+
+def run_oracle_sweep(a):
+    """The oracle's layer forward on the host cores for each workload: tokens/s on a bounded
+    token sample (about 3 s each), with the host's core count and CPU model."""
+    import platform
+
+    import torch
+
+    from deterministic_invariant_routing_b200 import synthetic
+
+    import oracle
+    gen = "cuda" if torch.cuda.is_available() else "cpu"  # weights drawn on the GPU if any
+    model = platform.processor()
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    cases = [("tiny", 64), ("dspark", 8192), ("qwen3_30b_a3b", 1), ("qwen3_30b_a3b", 64),
+             ("qwen3_30b_a3b", 4096), ("qwen3_30b_a3b", 16384), ("dsv_sigmoid", 8192)]
+    rows = []
+    for name, T in cases:
+        s, d = synthetic.make_layer(name, T=T, device=gen)
+        d = {k: (None if v is None else v.cpu()) for k, v in d.items()}
+        r = cpu_baseline(s, d, seconds=3.0)
+        del d
+        rows.append({"workload": f"{name}_T{T}", "tokens_per_s": r["value"],
+                     "sample": r["sample"]})
+    print(json.dumps({"oracle_sweep": "oracle layer forward on the host cores",
+                      "nproc": os.cpu_count(), "threads": oracle.num_threads(),
+                      "cpu_model": model, "rows": rows}), flush=True)
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return run_reference(a)
+    if a.sweep:
+        return run_sweep(a)
+    if a.oracle_sweep:
+        return run_oracle_sweep(a)
 
     import torch
     import torch.distributed as dist
@@ -378,7 +468,6 @@ def main():
         return reduce_max(v, dev, world)
 
     K = a.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
@@ -386,10 +475,19 @@ def main():
     with ClockSampler(gpu_id) as clk:
         start.record()
         for k in range(K):
-            layer(x, check=False, stage_events=ev[k])
+            layer(x, check=False)
         stop.record()
         barrier()
     ms = max_over_ranks(start.elapsed_time(stop) / K)
+    moe.check_status(layer.status)
+
+    # the stage split, in a separate pass: events recorded between the kernels break the
+    # dependent-launch overlap, so they stay out of the timed steps above
+    Ks = max(1, min(a.split_steps, K))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(Ks)]
+    for k in range(Ks):
+        layer(x, check=False, stage_events=ev[k])
+    barrier()
     moe.check_status(layer.status)
 
     def stage_ms(i, j):
@@ -443,6 +541,8 @@ def main():
                            "peaks": f"{pk_src}: {peak} TFLOP/s bf16 sustained, "
                                     f"{pk['hbm_gbs']} GB/s"},
         "stage_ms": stages,
+        "stage_split": f"separate pass of {Ks} steps with events between the kernels "
+                       f"({sum(stages.values()):.4f} ms per step there)",
         "e2e": {"value": job_tokens_per_s(s.T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
                 "ms_per_step": ms_e2e, "chunk_tokens": a.e2e_chunk,
