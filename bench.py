@@ -43,7 +43,7 @@ def parse():
     p.add_argument("--workload", default="qwen3_30b_a3b")
     p.add_argument("--T", type=int, default=16384)
     p.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
-    p.add_argument("--e2e-chunk", type=int, default=4096,
+    p.add_argument("--e2e-chunk", type=int, default=5120,
                    help="tokens per chunk of the host-memory call (copies overlap compute)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",

@@ -382,8 +382,59 @@ int forward_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* w_router,
     return rec(ev, 7, st);
 }
 
-// scratch of moe_forward_host: the forward workspace of one chunk, then two x chunks and
-// two out chunks (double buffering)
+// Token chunks of moe_forward_host for a nominal chunk C: up to 2 C tokens in chunks of at
+// most C (equal sizes); beyond that a first and a last chunk of C / 2 -- the pipeline's fill
+// (the first copy in) and drain (the last copy out) are only as long as those -- and the
+// tokens between them in equal chunks of at most 3 C / 2, since the layer runs faster per
+// token on more tokens. Start of chunk i = chunk_start(i), i = 0..n (chunk_start(n) = T).
+struct HostChunks {
+    int T, n, edge, mid_n, mid_base, mid_rem;
+    int64_t start(int i) const
+    {
+        if (edge == 0) {  // n equal chunks
+            const int64_t q = T / n, r = T % n;
+            return (int64_t)i * q + (i < r ? i : r);
+        }
+        if (i == 0) return 0;
+        if (i >= n) return T;
+        const int k = i - 1;  // middle chunks before chunk i
+        return edge + (int64_t)k * mid_base + (k < mid_rem ? k : mid_rem);
+    }
+    int64_t max_chunk() const
+    {
+        int64_t m = 0;
+        for (int i = 0; i < n; ++i) {
+            const int64_t len = start(i + 1) - start(i);
+            if (len > m) m = len;
+        }
+        return m;
+    }
+};
+
+HostChunks host_chunks(int T, int C)
+{
+    HostChunks h{};
+    h.T = T;
+    if (T <= 0) {
+        h.n = 0;
+        return h;
+    }
+    if (C < 2 || T <= 2 * (int64_t)C) {
+        h.n = (int)((T + (int64_t)C - 1) / C);
+        return h;
+    }
+    h.edge = C / 2;
+    const int64_t mid = T - 2 * (int64_t)h.edge;
+    const int64_t cap = (int64_t)C + C / 2;
+    h.mid_n = (int)((mid + cap - 1) / cap);
+    h.mid_base = (int)(mid / h.mid_n);
+    h.mid_rem = (int)(mid % h.mid_n);
+    h.n = h.mid_n + 2;
+    return h;
+}
+
+// scratch of moe_forward_host: the forward workspace of the largest chunk, then two x
+// chunks and two out chunks (double buffering)
 struct HostLayout {
     int chunk;
     size_t fwd, x_buf[2], out_buf[2], total;
@@ -392,7 +443,8 @@ struct HostLayout {
 HostLayout host_layout(const moe_cfg& c, int chunk_tokens)
 {
     HostLayout L{};
-    L.chunk = chunk_tokens < c.T ? chunk_tokens : (c.T > 0 ? c.T : 1);
+    const int64_t big = c.T > 0 ? host_chunks(c.T, chunk_tokens).max_chunk() : 1;
+    L.chunk = (int)(big > 0 ? big : 1);
     moe_cfg cc = c;
     cc.T = L.chunk;
     const size_t buf = up((size_t)L.chunk * c.H * 2);
@@ -892,18 +944,17 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
     HostPipe* hp = nullptr;
     if ((rc = cuda_rc(host_pipe(&hp))) != MOE_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int C = L.chunk;
+    const HostChunks hc = host_chunks(c.T, chunk_tokens);
     const size_t row_bytes = (size_t)c.H * 2;
     if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
     // the copy streams start after everything already queued on the caller's stream
     if ((rc = cuda_rc(cudaEventRecord(hp->start, st))) != MOE_OK) return rc;
     if ((rc = cuda_rc(cudaStreamWaitEvent(hp->in, hp->start, 0))) != MOE_OK) return rc;
     if ((rc = cuda_rc(cudaStreamWaitEvent(hp->out, hp->start, 0))) != MOE_OK) return rc;
-    const int n_chunks = (c.T + C - 1) / C;
-    for (int i = 0; i < n_chunks; ++i) {
+    for (int i = 0; i < hc.n; ++i) {
         const int slot = i & 1;
-        const int t0 = i * C;
-        const int tn = (c.T - t0) < C ? (c.T - t0) : C;
+        const int t0 = (int)hc.start(i);
+        const int tn = (int)(hc.start(i + 1) - t0);
         uint16_t* xb = at<uint16_t>(ws, L.x_buf[slot]);
         uint16_t* ob = at<uint16_t>(ws, L.out_buf[slot]);
         // H2D of chunk i once the compute of chunk i-2 no longer reads this x buffer

@@ -297,10 +297,12 @@ MOE_API int moe_router_stats(const moe_cfg* cfg, const float* logits, const uint
 /*
  * The whole layer from and to HOST memory, overlapping the transfers with the compute
  * (the chunked form is exact: results are bitwise independent of how tokens are split).
- * Tokens are processed in chunks of `chunk_tokens`: the host->device copy of chunk i+1 and
- * the device->host copy of chunk i-1 run on two library-owned copy streams while chunk i
- * runs on `stream`, double-buffered in `ws`. When `stream` completes, out_host holds the
- * result. Same output bits as moe_forward on the same tokens.
+ * Tokens are processed in chunks around a nominal `chunk_tokens` = C: up to 2 C tokens in
+ * equal chunks of at most C; beyond that a first and a last chunk of C / 2 (a short pipeline
+ * fill and drain) with equal chunks of at most 3 C / 2 between them. The host->device copy
+ * of chunk i+1 and the device->host copy of chunk i-1 run on two library-owned copy
+ * streams while chunk i runs on `stream`, double-buffered in `ws`. When `stream`
+ * completes, out_host holds the result. Same output bits as moe_forward on the same tokens.
  *
  *  x_host       [T,H] bf16 in HOST memory (page-locked for the copies to overlap).
  *  out_host     [T,H] bf16 in HOST memory (page-locked).
