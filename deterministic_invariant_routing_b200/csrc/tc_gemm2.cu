@@ -466,6 +466,10 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
         const uint32_t erow = (uint32_t)lane * 64u, eswz = ((uint32_t)lane >> 1) & 3u;
         // 32 x 32 block of rows [row_blk, +32), columns [col, +32): through shared memory
         // and TMA when the whole block is inside the group, else the valid rows directly
+        // fp32 weight gradients and the kept gate/up values are not read again soon: their
+        // lines go first when L2 needs room, ahead of the operands the tiles share
+        const uint64_t evict_first =
+            (EPI == EPI_WGRAD || EPI == EPI_SWIGLU_SAVE) ? l2_evict_first_policy() : 0ull;
         auto store_block = [&](const uint32_t (&pk)[16], bool full_blk, bool valid,
                                int row_blk, int col, uint16_t* dst_row,
                                const CUtensorMap* map) {
@@ -483,7 +487,10 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(map, b, col, row_blk);
+                    if (EPI == EPI_WGRAD || (EPI == EPI_SWIGLU_SAVE && map == &tmG))
+                        tma_store_2d_hint(map, b, col, row_blk, evict_first);
+                    else
+                        tma_store_2d(map, b, col, row_blk);
                     bulk_commit();
                 }
                 eb ^= 1u;
