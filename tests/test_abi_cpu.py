@@ -118,3 +118,28 @@ def test_binding_refuses_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(N, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         N.load()
+
+
+def test_host_chunk_schedule(lib):
+    """moe_forward_host's scratch is the forward workspace of its largest chunk plus two
+    input and two output buffers of that many rows: beyond 2 C tokens the first and last
+    chunks are C / 2 and the ones between are equal and at most 3 C / 2; up to 2 C the
+    chunks are equal and at most C."""
+    H = 2048
+    shape = dict(H=H, E=128, K=8, I=768)
+
+    def fwd(T):
+        return lib.moe_workspace_bytes(ctypes.byref(cfg(T=T, **shape)), N.MOE_STAGE_FORWARD)
+
+    def host(T, chunk):
+        return lib.moe_forward_host_workspace_bytes(ctypes.byref(cfg(T=T, **shape)), chunk)
+
+    def expect(largest):
+        return fwd(largest) + 4 * largest * H * 2
+
+    assert host(16384, 4096) == expect(6144)   # 2048 | 6144 6144 | 2048
+    assert host(16384, 5120) == expect(5632)   # 2560 | 5632 5632 | 2560
+    assert host(20000, 4096) == expect(5302)   # 2048 | 5302 5301 5301 | 2048
+    assert host(5000, 4096) == expect(2500)    # 2500 2500
+    assert host(3000, 4096) == expect(3000)    # one chunk
+    assert host(16384, 8192) == expect(8192)   # 8192 8192
