@@ -135,12 +135,24 @@ __device__ __forceinline__ PairTile decode_pair_tile(int t, int n_tiles, int gro
 
 // K-grouped products (EPI_WGRAD): group g owns K columns [k_offsets[g], k_offsets[g+1]);
 // tiles are (g, row tile, n), n fastest
-__device__ __forceinline__ PairTile decode_wgrad_tile(int t, const PairArgs& a)
+__device__ __forceinline__ PairTile decode_wgrad_tile(int t, const PairArgs& a,
+                                                     const int32_t* order, int nclusters,
+                                                     int total)
 {
-    PairTile ti;
+    // Tiles run in rounds of nclusters (cluster c takes tile c of every round). They are
+    // dealt by descending cost -- groups ordered by their K length, longest first -- and
+    // every other round in reverse cluster order, so that each cluster's total K is close
+    // to the mean however skewed the groups are. Only the schedule changes: a tile's
+    // arithmetic is the same wherever it runs.
     const int per = a.m_tiles * a.n_tiles;
-    ti.g = t / per;
-    const int rem = t - ti.g * per;
+    const int k = t / nclusters, j = t - k * nclusters;
+    const int base = k * nclusters;
+    const int n_here = total - base < nclusters ? total - base : nclusters;
+    const int s = base + ((k & 1) ? n_here - 1 - j : j);
+    const int r = s / per;
+    PairTile ti;
+    ti.g = order[r];
+    const int rem = s - r * per;
     const int mt = rem / a.n_tiles;
     ti.n = rem - mt * a.n_tiles;
     ti.row0 = (int64_t)mt * PM;
@@ -212,7 +224,19 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     }
     if (warp == 1) tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
     pdl_wait();  // the previous kernel's writes (offsets, operands) are visible from here on
-    if (warp == 2) {
+    if (warp == 2 && EPI == EPI_WGRAD) {
+        // groups by descending K length (ties: lower group first): order[rank] = group
+        int32_t* kl = offs;
+        int32_t* order = prefix;
+        for (int g = lane; g < G; g += 32) kl[g] = args.k_offsets[g + 1] - args.k_offsets[g];
+        __syncwarp();
+        for (int g = lane; g < G; g += 32) {
+            const int kg = kl[g];
+            int r = 0;
+            for (int h = 0; h < G; ++h) r += (kl[h] > kg || (kl[h] == kg && h < g)) ? 1 : 0;
+            order[r] = g;
+        }
+    } else if (warp == 2) {
         auto row_off = [&](int g) -> int {
             return args.offsets ? args.offsets[g] : (g == 0 ? 0 : args.rows);
         };
@@ -251,7 +275,7 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
         (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE);
     const int total = kWgrad ? G * args.m_tiles * args.n_tiles : prefix[G] * args.n_tiles;
     auto decode = [&](int t) -> PairTile {
-        if (kWgrad) return decode_wgrad_tile(t, args);
+        if (kWgrad) return decode_wgrad_tile(t, args, prefix, nclusters, total);
         return decode_pair_tile(t, args.n_tiles, G, prefix, offs, args.k_blocks);
     };
 
