@@ -31,8 +31,9 @@
 //
 // Output: each epilogue warp owns 32 accumulator rows and writes them 32 columns at a time.
 // Epilogues that move more global bytes per tile than the main loop hides (the fp32
-// outputs and the SwiGLU backward's gate/up reads) run two warps per 32 rows, each taking
-// every other 32-column chunk.
+// outputs, the SwiGLU backward's gate/up reads, and plain bf16 outputs, whose products
+// have the shortest K loops) run two warps per 32 rows, each taking every other 32-column
+// chunk.
 // A block whose 32 rows all lie inside the group goes through a 2 KiB shared-memory tile
 // (64-byte swizzle, two per warp, alternating) and one TMA store; the partial block at a
 // group's end is stored row by row from registers, so no padding row reaches global memory.
@@ -80,7 +81,9 @@ struct Cfg2 {
     // epilogue warps: two per TMEM lane quarter (each taking every other 32-column chunk)
     // where the epilogue moves more global bytes than the main loop hides with one
     static constexpr int kEpiWarps =
-        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD) ? 8 : 4;
+        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD || EPI == EPI_BF16)
+            ? 8
+            : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     // outputs go through two 2 KiB store tiles per epilogue warp (32 rows of 32 bf16 or 16
     // fp32 values); the router's fp32 logits are written from registers
