@@ -82,3 +82,25 @@ def test_single_process_defaults():
     import bench
     assert bench.reduce_max(3.5, "cpu", 1) == 3.5
     assert bench.job_tokens_per_s(16384, 1, 1.6) == pytest.approx(16384 / 1.6e-3)
+
+
+def test_reference_arm_line_on_cpu():
+    """`bench.py --impl reference` times the oracle on the host and prints one JSON line with
+    the reference arm's keys (no GPU needed)."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--T", "64", "--steps", "1", "--warmup", "1"], cwd=root,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == "tiny_T64"
