@@ -30,10 +30,9 @@
 // recorded in MOE_ST_PIPE_TIMEOUT.
 //
 // Output: each epilogue warp owns 32 accumulator rows and writes them 32 columns at a time.
-// Epilogues that move more global bytes per tile than the main loop hides (the fp32
-// outputs, the SwiGLU backward's gate/up reads, and plain bf16 outputs, whose products
-// have the shortest K loops) run two warps per 32 rows, each taking every other 32-column
-// chunk.
+// Every epilogue but the router's fp32 one runs two warps per 32 rows, each taking every
+// other 32-column chunk, so that storing a tile's outputs (and, for the SwiGLU backward,
+// reading its gate/up values) keeps pace with the next tile's main loop.
 // A block whose 32 rows all lie inside the group goes through a 2 KiB shared-memory tile
 // (64-byte swizzle, two per warp, alternating) and one TMA store; the partial block at a
 // group's end is stored row by row from registers, so no padding row reaches global memory.
@@ -81,7 +80,8 @@ struct Cfg2 {
     // epilogue warps: two per TMEM lane quarter (each taking every other 32-column chunk)
     // where the epilogue moves more global bytes than the main loop hides with one
     static constexpr int kEpiWarps =
-        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD || EPI == EPI_BF16)
+        (EPI == EPI_DSWIGLU || EPI == EPI_SWIGLU_SAVE || EPI == EPI_WGRAD || EPI == EPI_BF16 ||
+         EPI == EPI_SWIGLU)
             ? 8
             : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
