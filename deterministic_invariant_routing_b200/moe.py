@@ -385,11 +385,12 @@ def forward_host_workspace_bytes(cfg: Config, chunk: int) -> int:
 
 
 def forward_host(cfg: Config, x_host, w_router, w13, w2, logit_bias=None, sel_bias=None,
-                 token_mask=None, w13_s=None, w2_s=None, out_host=None, chunk: int = 4096,
+                 token_mask=None, w13_s=None, w2_s=None, out_host=None, chunk: int = 5120,
                  ws=None, status=None, check: bool = True):
     """The layer from and to host memory in one C-ABI call, transfers overlapped with the
-    compute in chunks of `chunk` tokens. x_host / out_host are CPU bf16 tensors (pin them
-    for the overlap); weights, biases and the mask are on the device."""
+    compute in chunks around `chunk` tokens (half-size first and last chunks, middle ones of
+    at most 1.5 x chunk; see moe_forward_host). x_host / out_host are CPU bf16 tensors (pin
+    them for the overlap); weights, biases and the mask are on the device."""
     dev = w13.device
     T, H, E, K, I, Is = cfg.T, cfg.H, cfg.E, cfg.K, cfg.I, cfg.I_shared
     cpu = torch.device("cpu")
@@ -431,7 +432,7 @@ class MoELayer:
         self.ws = _ws(workspace_bytes(cfg.with_T(self.max_T), N.MOE_STAGE_FORWARD), dev, None)
         self.status = new_status(dev)
 
-    def forward_host(self, x_host, out_host=None, chunk: int = 4096, token_mask=None,
+    def forward_host(self, x_host, out_host=None, chunk: int = 5120, token_mask=None,
                      check=True):
         """The layer from pinned host memory to pinned host memory (see forward_host)."""
         T = x_host.shape[0]
