@@ -143,3 +143,64 @@ def test_host_chunk_schedule(lib):
     assert host(5000, 4096) == expect(2500)    # 2500 2500
     assert host(3000, 4096) == expect(3000)    # one chunk
     assert host(16384, 8192) == expect(8192)   # 8192 8192
+
+
+def test_training_and_extra_entry_points_reject_bad_arguments(lib):
+    """The backward, the training forward, the order-invariant combine, the router statistics
+    and the host-buffer forward validate their arguments on the host before any device work
+    (each failing call below returns before a CUDA call is made)."""
+    c = cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    need_b = lib.moe_workspace_bytes(ctypes.byref(c), N.MOE_STAGE_BACKWARD)
+    assert need_b > 0
+
+    def bwd(**over):
+        names = ["x", "w_router", "token_mask", "w13", "w2", "w13_s", "w2_s", "logits",
+                 "topk_ids", "topk_w", "dout", "dx", "dw_router", "dw13", "dw2", "dw13_s",
+                 "dw2_s", "d_topk_w", "dlogits"]
+        p = {n: fake for n in names}
+        p.update(token_mask=None, w13_s=None, w2_s=None, dw13_s=None, dw2_s=None)
+        p.update({k: v for k, v in over.items() if k in names})
+        return lib.moe_backward(ctypes.byref(over.get("cfg", c)), *[p[n] for n in names],
+                                over.get("saved", 0), fake, fake, over.get("ws_bytes", need_b),
+                                None)
+
+    assert bwd(saved=2) == N.MOE_ERR_ARG
+    assert bwd(w13=None) == N.MOE_ERR_ARG
+    assert bwd(x=odd) == N.MOE_ERR_ARG
+    assert bwd(dw13=odd) == N.MOE_ERR_ARG
+    assert bwd(ws_bytes=need_b - 1) == N.MOE_ERR_WORKSPACE
+    cs = cfg(I_shared=256)
+    assert bwd(cfg=cs) == N.MOE_ERR_ARG  # a shared expert needs its weights and gradients
+    assert bwd(cfg=cfg(H=100)) == N.MOE_ERR_SHAPE
+
+    def ftrain(**over):
+        names = ["x", "w_router", "logit_bias", "sel_bias", "token_mask", "w13", "w2", "w13_s",
+                 "w2_s", "out", "logits", "topk_ids", "topk_w", "status", "ws"]
+        p = {n: fake for n in names}
+        p.update(logit_bias=None, sel_bias=None, token_mask=None, w13_s=None, w2_s=None)
+        p.update(over)
+        return lib.moe_forward_train(ctypes.byref(c), *[p[n] for n in names],
+                                     need_b if "ws_bytes" not in over else over["ws_bytes"], None)
+
+    assert ftrain(logits=None) == N.MOE_ERR_ARG
+    assert ftrain(topk_w=odd) == N.MOE_ERR_ARG
+    assert ftrain(out=None) == N.MOE_ERR_ARG
+
+    assert lib.moe_combine_invariant(ctypes.byref(c), None, fake, fake, None, None, fake,
+                                     None) == N.MOE_ERR_ARG
+    assert lib.moe_combine_invariant(ctypes.byref(c), fake, fake, fake, odd, None, fake,
+                                     None) == N.MOE_ERR_ARG
+
+    need_s = lib.moe_workspace_bytes(ctypes.byref(c), N.MOE_STAGE_STATS)
+    assert lib.moe_router_stats(ctypes.byref(c), fake, None, fake, fake, fake, None, fake, need_s,
+                                None) == N.MOE_ERR_ARG
+    assert lib.moe_router_stats(ctypes.byref(c), fake, None, fake, fake, fake, fake, fake,
+                                need_s - 1, None) == N.MOE_ERR_WORKSPACE
+
+    need_h = lib.moe_forward_host_workspace_bytes(ctypes.byref(c), 32)
+    assert lib.moe_forward_host(ctypes.byref(c), fake, fake, None, None, None, fake, fake, None,
+                                None, fake, fake, 0, fake, need_h, None) == N.MOE_ERR_ARG
+    assert lib.moe_forward_host(ctypes.byref(c), fake, fake, None, None, None, fake, fake, None,
+                                None, fake, fake, 32, fake, need_h - 1, None) == N.MOE_ERR_WORKSPACE
