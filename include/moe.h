@@ -325,7 +325,8 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
  * Train-Inference Consistency Roadmap", "Why DSV4 Flash MoE Drifts More Easily" and the
  * DSV4-WS1-2 row of "Follow-Up Issue Buckets"; the pages give no backward arithmetic).
  * Gradients of sum(dout * out) for the routes of the forward (selection has no gradient).
- * The forward intermediates are recomputed from x with the forward's kernels (same bits).
+ * The forward intermediates (dispatch, h, y and the fp32 gate/up values) are recomputed from
+ * x with the forward's kernels (same bits), or taken from `ws` after moe_forward_train.
  *
  *  Inputs (DEVICE): x, w_router, token_mask (or NULL), w13, w2, w13_s/w2_s as in
  *    moe_forward; logits [T,E] fp32, topk_ids [T,K], topk_w [T,K] as the forward returned
@@ -339,14 +340,15 @@ MOE_API int moe_forward_host(const moe_cfg* cfg, const uint16_t* x_host, const u
  *    d_topk_w[t,j] = dot32(dout_t, y_row): lane L of 32 sums the rounded products of the
  *      8-element chunks L, L+32, ... in order, then butterfly levels 16..1 (fp32);
  *    dy_row = bf16(topk_w[t,j] * dout_t); dy_shared = dout (0 for masked tokens);
- *    dh = bf16(dy . W2_e); [dg | du] = bf16(dh * u * silu'(g) | dh * silu(g)) with g, u the
- *      recomputed fp32 gate/up products; dx_row = bf16([dg | du] . W13_e);
+ *    dh = dy . W2_e kept in fp32; [dg | du] = bf16(dh * u * silu'(g) | dh * silu(g)) with
+ *      g, u the forward's fp32 gate/up products; dx_row = bf16([dg | du] . W13_e);
  *    dlogits: through the renormalisation and the score function in fp32, each operation
  *      rounded to nearest, rank-order sums (see the router backward of the oracle);
  *    dx_t = bf16(rank-order sum of dx_row + shared term + bf16(dlogits_t) . W_router), +0
  *      for masked tokens;
  *    dW = sum over an expert's rows, ascending, of dy^T h / [dg|du]^T x (fp32 accumulation
- *      on the tensor cores, bf16 operands); dW_router = sum_t bf16(dlogits_t)^T x_t.
+ *      on the tensor cores, bf16 operands); dW_router = sum over fixed token chunks (a
+ *      function of E, H and T), in chunk order, of the chunks' sums of bf16(dlogits_t)^T x_t.
  *  saved  0: the forward intermediates are recomputed from x; 1: `ws` holds those that
  *         moe_forward_train wrote for the same cfg, inputs and routes (not checked).
  *  ws  moe_workspace_bytes(cfg, MOE_STAGE_BACKWARD) bytes.
