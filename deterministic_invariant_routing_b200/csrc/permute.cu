@@ -10,8 +10,6 @@
 // block's base row per expert) -> placement (per-warp ranks from __match_any_sync in
 // assignment order). All integer, no floating point, no order-dependent atomics (the
 // only atomics are shared-memory histogram increments, whose sum is order-free).
-#include <mutex>
-
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -225,22 +223,15 @@ cudaError_t launch_permute(const moe_cfg& c, const int32_t* ids, int32_t* offset
 
 cudaError_t permute_fixed_scratch(int32_t** out)
 {
-    // In host code g_permute_scratch is only a stand-in symbol, not a device address:
-    // the address is asked of the runtime once per device, with that device current.
-    static std::mutex mu;
-    static int32_t* addr[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    // In host code g_permute_scratch is only a stand-in symbol, not a device address. The
+    // runtime is asked for the address on every call, with the caller's device current: a
+    // host-side lookup that allocates nothing, and that stays right when a device reset or
+    // a new primary context has moved the module since the previous call (a cached address
+    // would then point at freed memory).
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_permute_scratch);
-        if (e != cudaSuccess) return e;
-        addr[dev] = static_cast<int32_t*>(p);
-    }
-    *out = addr[dev];
+    *out = static_cast<int32_t*>(p);
     return cudaSuccess;
 }
 

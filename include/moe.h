@@ -145,6 +145,13 @@ MOE_API size_t moe_workspace_bytes(const moe_cfg* cfg, int stage);
  *  status     int32[MOE_STATUS_WORDS] device, cleared then counted; may be NULL.
  * Score arithmetic is the FP32 contract: exp_rl, the 32-lane softmax tree, IEEE
  * round-to-nearest adds/multiplies/divides, no FMA contraction outside exp_rl.
+ * Degenerate rows fail closed through the status words rather than by a made-up value:
+ * a softmax row whose logits are all -inf (or that holds a NaN) has no defined
+ * distribution -- its max is -inf, so every l - max is NaN -- and every score is NaN;
+ * the row counts once in MOE_ST_NAN_TOKENS, NaN keys rank below every number so it
+ * takes ids 0..K-1 by the tie rule, and its weights are NaN. A sigmoid or sqrtsoftplus
+ * row of all -inf has scores +0: it takes ids 0..K-1, a renormalised row counts in
+ * MOE_ST_ZERO_DENOM and its weights are 0.
  */
 MOE_API int moe_route(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
                       const float* logit_bias, const float* sel_bias,
@@ -183,8 +190,10 @@ MOE_API int moe_permute(const moe_cfg* cfg, const int32_t* topk_ids, const uint1
  *
  *  Limit: ceil(T*K / 2048) * E <= 262144 (e.g. E = 128 allows T*K <= 4,194,304); larger
  *         requests return MOE_ERR_WORKSPACE before anything is enqueued.
- *  The first call on a device looks up the array's device address (once per device, with
- *  that device current); make that first call before any stream capture.
+ *  Every call looks up the array's device address on the caller's current device (a
+ *  host-side query that allocates nothing), so a device reset or a new primary context
+ *  between calls does not leave a stale address behind. The first call on a device may
+ *  load the library's device code there: make that first call before any stream capture.
  *  All calls share the array and it keeps the last call's contents; nothing in it needs
  *  to start at zero (every call overwrites what it reads). Calls that overlap on the GPU
  *  (other streams, other host threads) race on it: serialise them.

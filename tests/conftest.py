@@ -47,3 +47,15 @@ def golden():
             return fix(json.load(f))
 
     return load
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """The parity report (level-2 errors, near-tie counts) of the tests that ran."""
+    try:
+        from helpers import REPORT
+    except Exception:  # pragma: no cover
+        return
+    if REPORT:
+        terminalreporter.write_sep("-", "parity report")
+        for line in REPORT:
+            terminalreporter.write_line(line)

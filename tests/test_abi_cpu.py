@@ -204,3 +204,25 @@ def test_training_and_extra_entry_points_reject_bad_arguments(lib):
                                 None, fake, fake, 0, fake, need_h, None) == N.MOE_ERR_ARG
     assert lib.moe_forward_host(ctypes.byref(c), fake, fake, None, None, None, fake, fake, None,
                                 None, fake, fake, 32, fake, need_h - 1, None) == N.MOE_ERR_WORKSPACE
+
+
+def test_permute_noalloc_size_limit(lib):
+    """moe_permute_noalloc serves ceil(T*K / 2048) * E <= 262144 histogram ints from its
+    fixed array: exactly at the limit the request passes the size check (it then stops at
+    the device check on a machine without a GPU), one assignment past it is refused with
+    MOE_ERR_WORKSPACE before anything else happens."""
+    import torch
+    fake = ctypes.c_void_p(1 << 20)
+
+    def call(**over):
+        c = cfg(**over)
+        return lib.moe_permute_noalloc(ctypes.byref(c), fake, None, fake, fake, fake, None,
+                                       None, None)
+
+    # E = 128, K = 8: 2048 blocks of 2048 assignments -> 2048 * 128 = 262144 ints
+    assert call(T=1 + (2048 * 2048) // 8, E=128, K=8) == N.MOE_ERR_WORKSPACE
+    assert call(T=600_000, E=1024, K=16) == N.MOE_ERR_WORKSPACE
+    if torch.cuda.is_available():
+        pytest.skip("the accepted edge would launch on the fake pointers")
+    assert call(T=(2048 * 2048) // 8, E=128, K=8) == N.MOE_ERR_DEVICE
+    assert call(T=1, E=1024, K=16) == N.MOE_ERR_DEVICE

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from deterministic_invariant_routing_b200 import moe, synthetic
-from helpers import DEV, bits, near_tie_count
+from helpers import DEV, REPORT, bits, near_tie_count
 
 pytestmark = pytest.mark.gpu
 
@@ -72,8 +72,9 @@ def test_batch_size_sweep(sweep):
             got = sweep.pick(sweep.run(x), pos)
         same(got, ref, f"batch {B}")
     lg = ref["logits"].cpu().numpy()
-    print(f"\nnear ties among the {sweep.n} targets (K-th vs K+1-th choice within 1 ulp): "
-          f"{near_tie_count(lg, sweep.s)}")
+    REPORT.append(f"level 3 batch sweep {BATCHES[0]}..{BATCHES[-1]}: {sweep.n} target tokens "
+                  f"bit-identical in {len(BATCHES)} batch sizes; near ties among them (K-th vs "
+                  f"K+1-th choice within 1 ulp): {near_tie_count(lg, sweep.s)}")
 
 
 @pytest.mark.parametrize("masked", [True, False])

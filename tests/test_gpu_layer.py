@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from deterministic_invariant_routing_b200 import moe, synthetic
-from helpers import (DEV, LEVEL2_ROW_REL, bits, expert_subset, layer, mean_abs_err,
+from helpers import (DEV, LEVEL2_ROW_REL, REPORT, bits, expert_subset, layer, mean_abs_err,
                      near_tie_count, reference_rows, row_rel_err)
 
 pytestmark = pytest.mark.gpu
@@ -114,9 +114,16 @@ def check_layer(name, T, n_sample=16, keep=None, report=None, **over):
     assert np.array_equal(bits(out1), bits(r["out"]))
     assert np.array_equal(bits(b["logits"]), bits(r["logits"]))
     assert np.array_equal(b["topk_ids"].cpu().numpy(), g_ids)
+    rep = dict(max_row_rel=float(errs[live].max()) if live.any() else 0.0,
+               mean_abs=mean_abs_err(g_out, ref), tokens=int(sel.size),
+               near_ties=near_tie_count(g_logits[sel], s, sb))
+    REPORT.append(f"level 2 {name} T={T}{'' if keep is None else f' keep={keep}'}"
+                  f"{''.join(f' {k}={v}' for k, v in over.items())}: "
+                  f"max row rel err {rep['max_row_rel']:.3e}, mean abs err "
+                  f"{rep['mean_abs']:.3e} over {rep['tokens']} sampled tokens, "
+                  f"{rep['near_ties']} near ties among them")
     if report is not None:
-        report.update(max_row_rel=float(errs.max()), mean_abs=mean_abs_err(g_out, ref),
-                      near_ties=near_tie_count(g_logits[sel], s, sb))
+        report.update(rep)
     return r
 
 
@@ -139,6 +146,54 @@ def test_tiny_ragged():
 @pytest.mark.parametrize("T", [1, 64, 4096, 16384])
 def test_qwen3_30b_a3b_shape(T):
     check_layer("qwen3_30b_a3b", T, n_sample=16)
+
+
+def expert_edge_rows(off):
+    """Per expert: its first and last row, every row of its last partial 32-row block
+    (stored from registers, not through a TMA store tile) and every row of a short tail of
+    1..128 rows past its last full 256-row tile (computed by the one-SM tail kernel)."""
+    rows = set()
+    for e in range(off.size - 1):
+        a, n = int(off[e]), int(off[e + 1] - off[e])
+        if n == 0:
+            continue
+        rows |= {a, a + n - 1}
+        rows |= set(range(a + n - n % 32, a + n))
+        if 0 < n % 256 <= 128:
+            rows |= set(range(a + n - n % 256, a + n))
+    return np.array(sorted(rows), np.int64)
+
+
+def test_qwen3_30b_a3b_expert_edge_rows_T16384():
+    """Level 2 at the bench size on the rows where a kernel's bookkeeping could go wrong
+    without a sampled row noticing: every expert's first and last row, its partial 32-row
+    block and its short tail (see expert_edge_rows), each expert output row against the
+    FP64 expert FFN of its token (row max relative error <= 1e-2)."""
+    from oracle import backward64 as B
+    T = 16384
+    s, d, cfg = layer("qwen3_30b_a3b", T)
+    r = run_stages(cfg, d)
+    off = r["offsets"].cpu().numpy()
+    perm = r["perm_token"].cpu().numpy()
+    rows = expert_edge_rows(off)
+    x64 = B.bf16_to_f64(bits(d["x"]))
+    y_g = r["y"].float().cpu().numpy().astype(np.float64)
+    worst, n_tail, errs = 0.0, 0, []
+    for e in range(s.E):
+        rr = rows[(rows >= off[e]) & (rows < off[e + 1])]
+        if rr.size == 0:
+            continue
+        n = int(off[e + 1] - off[e])
+        n_tail += (n % 256) if 0 < n % 256 <= 128 else 0
+        _, _, _, y64 = B._experts_forward(x64[perm[rr]], B.bf16_to_f64(bits(d["w13"][e])),
+                                          B.bf16_to_f64(bits(d["w2"][e])))
+        rel = np.abs(y_g[rr] - y64).max(axis=1) / np.abs(y64).max(axis=1)
+        assert np.all(rel <= LEVEL2_ROW_REL), (e, rr[np.argmax(rel)], rel.max())
+        errs.append(np.abs(y_g[rr] - y64).mean())
+        worst = max(worst, float(rel.max()))
+    REPORT.append(f"level 2 qwen3_30b_a3b T={T} expert edge rows: {rows.size} rows "
+                  f"({n_tail} in short tails) max row rel err {worst:.3e}, mean abs err "
+                  f"{float(np.mean(errs)):.3e}")
 
 
 def test_qwen3_30b_a3b_masked():

@@ -16,7 +16,8 @@ SM, SG, SP = moe.SOFTMAX, moe.SIGMOID, moe.SQRTSOFTPLUS
 
 def adversarial_logits(T, E, seed, std=3.0):
     """Random logits with injected exact ties (at every rank), all-equal rows, signed
-    zeros, -inf, a NaN row and a wide dynamic range (exp_rl's full input domain)."""
+    zeros, -inf, a NaN row, a row of only -inf and a wide dynamic range (exp_rl's full
+    input domain)."""
     l = synthetic.random_logits(T, E, seed, std=std).numpy()
     rng = np.random.default_rng(seed)
     for t in range(0, min(T, 40)):
@@ -29,6 +30,8 @@ def adversarial_logits(T, E, seed, std=3.0):
         l[43, : max(1, E // 2)] = -np.inf
         l[44] = rng.uniform(-80, 80, E)
         l[45, rng.integers(0, E)] = np.nan
+    if T > 46:
+        l[46] = -np.inf                   # no defined softmax: NaN scores, fails closed
     return np.ascontiguousarray(l.astype(np.float32))
 
 

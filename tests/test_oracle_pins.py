@@ -276,6 +276,25 @@ def test_route_mask_and_zero_denominator():
     assert st[0] == 1 and list(ids[0]) == [0, 1] and np.all(np.isnan(w))
 
 
+def test_route_all_minus_inf_row_fails_closed():
+    """A row whose logits are all -inf has no softmax (max = -inf, every l - max is NaN):
+    every score is NaN, the row is counted once as a NaN token and takes ids 0..K-1 by the
+    tie rule with NaN weights. Sigmoid and sqrtsoftplus scores of -inf are exactly +0:
+    ids 0..K-1, the renormalisation denominator is 0, weights 0, counted there instead."""
+    l = np.full((3, 8), -np.inf, F32)
+    l[1, 6] = 0.0                          # one finite logit: p = 1 on expert 6
+    s = oracle.scores_fp32(l[0], oracle.SOFTMAX)
+    assert np.all(np.isnan(s))
+    ids, w, st = oracle.route_fp32(l, 3, oracle.SOFTMAX, True)
+    assert list(st) == [2, 0]
+    assert list(ids[0]) == [0, 1, 2] and np.all(np.isnan(w[0]))
+    assert list(ids[1]) == [6, 0, 1] and list(w[1]) == [1.0, 0.0, 0.0]
+    for fn in (oracle.SIGMOID, oracle.SQRTSOFTPLUS):
+        assert np.all(oracle.scores_fp32(l[0], fn) == 0.0)
+        ids, w, st = oracle.route_fp32(l[[0, 2]], 3, fn, True)
+        assert list(st) == [0, 2] and np.all(ids == [0, 1, 2]) and np.all(w == 0.0)
+
+
 # ------------------------------------------------------------------ permutation
 
 def test_permute_properties():
