@@ -71,6 +71,7 @@ SIGNATURES = {
     "moe_forward_host": (_I, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_abi_version": (_I, []),
+    "moe_pipeline_wait_selftest": (_I, [_P, ctypes.c_longlong, _P]),
 }
 
 _lock = threading.Lock()

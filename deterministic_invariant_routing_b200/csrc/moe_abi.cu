@@ -727,7 +727,18 @@ using namespace moe;
 
 extern "C" {
 
-MOE_API int moe_abi_version(void) { return 103; }
+MOE_API int moe_abi_version(void) { return 104; }
+
+MOE_API int moe_pipeline_wait_selftest(int32_t* status, long long limit_cycles, void* stream)
+{
+    if (status == nullptr) return MOE_ERR_ARG;
+    if (limit_cycles < 1000 || limit_cycles > 2000000000LL) return MOE_ERR_ARG;
+    int rc;
+    if ((rc = check_device()) != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    return cuda_rc(launch_pipe_wait_selftest(status, limit_cycles, st));
+}
 
 MOE_API const char* moe_status_string(int code)
 {

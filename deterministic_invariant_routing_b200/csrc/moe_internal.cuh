@@ -173,6 +173,9 @@ struct RouterProblem {
 };
 cudaError_t launch_router(const RouterProblem& p, cudaStream_t st);
 
+// diagnostic: one bounded pipeline wait that runs out (see moe_pipeline_wait_selftest)
+cudaError_t launch_pipe_wait_selftest(int32_t* status, long long limit_cycles, cudaStream_t st);
+
 // device facts
 int num_sms();
 bool device_is_sm100();

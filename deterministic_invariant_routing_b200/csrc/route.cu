@@ -37,9 +37,37 @@ __device__ __forceinline__ int warp_argmax_id(unsigned long long k)
     return (int)(0xffffffffu - mlo);
 }
 
-// NE = experts held per lane (E <= 32 * NE)
+// descending sort of a lane's keys: the optimal 5-exchange network for 4, odd-even
+// transposition otherwise (the order of equal keys cannot matter: keys are distinct)
 template <int NE>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
+__device__ __forceinline__ void sort_desc(unsigned long long (&key)[NE])
+{
+    auto cx = [&](int a, int b) {
+        const unsigned long long ka = key[a], kb = key[b];
+        const bool swap = ka < kb;
+        key[a] = swap ? kb : ka;
+        key[b] = swap ? ka : kb;
+    };
+    if constexpr (NE == 4) {
+        cx(0, 1);
+        cx(2, 3);
+        cx(0, 2);
+        cx(1, 3);
+        cx(1, 2);
+    } else {
+#pragma unroll
+        for (int pass = 0; pass < NE; ++pass) {
+#pragma unroll
+            for (int i = pass & 1; i + 1 < NE; i += 2) cx(i, i + 1);
+        }
+    }
+}
+
+// NE = experts held per lane (E <= 32 * NE)
+// up to 128 experts the kernel fits 40 registers (6 resident blocks of 8 warps per SM):
+// its K selection rounds are a chain of warp reductions, so latency is hidden by warps
+template <int NE>
+__global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const float* __restrict__ logits, int T, int E,
                                                     int K, const float* __restrict__ sel_bias,
                                                     const uint8_t* __restrict__ mask, int score_fn,
                                                     int renorm, float route_scale,
@@ -108,41 +136,33 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                 if (e < E && ((kept >> (e / gs)) & 1u) == 0u) key[i] = 0ull;
             }
         }
-        // each lane orders its own keys (descending, scores alongside) once; then K rounds
-        // of a warp arg-max over the lanes' heads, the winning lane dropping its head
-        float sv[NE];
-#pragma unroll
-        for (int i = 0; i < NE; ++i) sv[i] = s[i];
-#pragma unroll
-        for (int pass = 0; pass < NE; ++pass) {
-#pragma unroll
-            for (int i = pass & 1; i + 1 < NE; i += 2) {
-                const bool swap = key[i] < key[i + 1];
-                const unsigned long long k0 = key[i], k1 = key[i + 1];
-                const float s0 = sv[i], s1 = sv[i + 1];
-                key[i] = swap ? k1 : k0;
-                key[i + 1] = swap ? k0 : k1;
-                sv[i] = swap ? s1 : s0;
-                sv[i + 1] = swap ? s0 : s1;
-            }
-        }
+        // each lane orders its own keys (descending) once; then K rounds of a warp arg-max
+        // over the lanes' heads, the winning lane dropping its head. Lane j keeps the id
+        // of round j; the scores stay where the lanes computed them and are fetched once.
+        sort_desc<NE>(key);
         int my_id = -1;
-        float my_s = 0.0f, den = 0.0f;
         for (int j = 0; j < K; ++j) {
             const int e = warp_argmax_id(key[0]);
-            const int owner = e & 31;
-            const float se = __shfl_sync(0xffffffffu, sv[0], owner);
-            if (lane == owner) {
+            if (lane == (e & 31)) {
 #pragma unroll
-                for (int i = 0; i + 1 < NE; ++i) {
-                    key[i] = key[i + 1];
-                    sv[i] = sv[i + 1];
-                }
+                for (int i = 0; i + 1 < NE; ++i) key[i] = key[i + 1];
                 key[NE - 1] = 0ull;
             }
-            den = (j == 0) ? se : __fadd_rn(den, se);
-            if (lane == j) { my_id = e; my_s = se; }
+            if (lane == j) my_id = e;
         }
+        // the unbiased score of this lane's pick: slot my_id / 32 of lane my_id % 32
+        float my_s = 0.0f;
+        {
+            const int src = my_id & 31, slot = my_id >> 5;
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                const float v = __shfl_sync(0xffffffffu, s[i], src);
+                if (i == slot) my_s = v;
+            }
+        }
+        // renormalisation denominator: the picks' scores added in rank order
+        float den = __shfl_sync(0xffffffffu, my_s, 0);
+        for (int j = 1; j < K; ++j) den = __fadd_rn(den, __shfl_sync(0xffffffffu, my_s, j));
         if (renorm && den == 0.0f) zero_den += (lane == 0);
         if (lane < K) {
             float wv;
@@ -167,10 +187,11 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bi
 {
     const int threads = 256, wpb = threads / 32;
     int blocks = (c.T + wpb - 1) / wpb;
-    const int cap = num_sms() * 8;
-    if (blocks > cap) blocks = cap;
     const int n_group = c.n_group > 1 ? c.n_group : 0;
     const size_t smem = n_group ? (size_t)wpb * c.E * sizeof(float) : 0;
+    // one wave of resident blocks, each warp taking every (grid warps)-th token
+    const int cap = resident_blocks((const void*)route_kernel<NE>, threads, smem);
+    if (blocks > cap) blocks = cap;
     return launch_pdl(route_kernel<NE>, dim3(blocks), dim3(threads), smem, st, logits, c.T, c.E,
                       c.K, sel_bias, mask, c.score_fn, c.renorm, c.route_scale, n_group,
                       c.topk_group, ids, w, status);

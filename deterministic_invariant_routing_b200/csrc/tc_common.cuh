@@ -12,7 +12,10 @@ namespace {
 
 constexpr int BK = 64;                              // k-block: one 128-byte swizzle row
 constexpr long long kTimeoutCycles = 2000000000LL;  // about a second at B200 clocks
-constexpr int kSmemBudget = 196608;                 // bytes for the operand ring
+#ifndef MOE_SMEM_BUDGET
+#define MOE_SMEM_BUDGET 196608
+#endif
+constexpr int kSmemBudget = MOE_SMEM_BUDGET;        // bytes for the operand ring
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -55,7 +58,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 // is out of line; wait_bounded() below tests the barrier inline first.
 __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, int32_t* status,
-                                               bool honour_abort)
+                                               bool honour_abort,
+                                               long long limit = kTimeoutCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -63,7 +67,7 @@ __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0u) {
             if (honour_abort && *abort_flag) return false;
-            if (clock64() - t0 > kTimeoutCycles) {
+            if (clock64() - t0 > limit) {
                 if (!*abort_flag) {
                     *abort_flag = 1;
                     status_add(status, MOE_ST_PIPE_TIMEOUT, 1);

@@ -258,7 +258,29 @@ cudaError_t launch_router_variant(const RouterProblem& p, cudaStream_t st)
     return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, st, ma, mb, a);
 }
 
+// One CTA whose thread 0 waits, through the pipelines' bounded wait, on an mbarrier that
+// nothing arrives on: after `limit` cycles the wait gives up, raises the CTA's abort flag
+// and counts MOE_ST_PIPE_TIMEOUT, as a stuck stage of a tensor-core pipeline would. No
+// copy, MMA or tensor memory is involved, so giving up leaves nothing in flight.
+__global__ void pipe_wait_selftest_kernel(int32_t* status, long long limit)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        wait_bounded_slow(smem_u32(&bar), 0u, &abort_flag, status, true, limit);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_pipe_wait_selftest(int32_t* status, long long limit_cycles, cudaStream_t st)
+{
+    pipe_wait_selftest_kernel<<<1, 32, 0, st>>>(status, limit_cycles);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_router(const RouterProblem& p, cudaStream_t st)
 {

@@ -221,6 +221,18 @@ def combine(cfg: Config, y, topk_w, dest_row, y_shared=None, token_mask=None,
     return out
 
 
+def pipeline_wait_selftest(dev, limit_cycles: int = 1_000_000, check: bool = True):
+    """Run one bounded pipeline wait that nothing satisfies (moe_pipeline_wait_selftest):
+    it gives up after limit_cycles and counts a pipeline timeout in the returned status
+    words; with check=True the count raises StatusError, as in any other call."""
+    st = new_status(dev)
+    _rc(N.load().moe_pipeline_wait_selftest(_p(st), int(limit_cycles), _stream(st.device)),
+        "moe_pipeline_wait_selftest")
+    if check:
+        check_status(st)
+    return st
+
+
 def router_stats(cfg: Config, logits, offsets, token_mask=None):
     """Router statistics of a routed batch: {tokens_per_expert [E] int32, mean_prob [E]
     fp32, aux [1] fp32} (the load-balance value E * sum_e load_e * mean_prob_e, K when

@@ -390,6 +390,21 @@ MOE_API const char* moe_status_string(int code);
 /* ABI version of this header (major * 100 + minor). */
 MOE_API int moe_abi_version(void);
 
+/*
+ * Diagnostic of the fail-closed path ("DSV4 Flash MoE Train-Inference Consistency
+ * Roadmap", Follow-Up Issue Buckets: mismatches fail closed). Every pipeline wait of the
+ * library's tensor-core and staged-copy kernels is bounded; when one runs out, the kernel
+ * stops issuing work, drains what it has in flight, frees its tensor memory, counts
+ * MOE_ST_PIPE_TIMEOUT and returns. This call runs that bounded wait once, in a one-CTA
+ * kernel, on an mbarrier that nothing arrives on, with the limit shortened to
+ * limit_cycles (1000 .. 2e9 SM clock cycles; the kernels use about 2e9): the wait gives up
+ * and status[MOE_ST_PIPE_TIMEOUT] becomes 1 instead of the GPU hanging. Nothing else is
+ * in flight in that kernel, so it cannot leave the device in a bad state.
+ *  status  int32[MOE_STATUS_WORDS] device, cleared first.
+ * Returns MOE_ERR_ARG for a NULL status or a limit out of range.
+ */
+MOE_API int moe_pipeline_wait_selftest(int32_t* status, long long limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

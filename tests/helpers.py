@@ -88,64 +88,127 @@ def near_tie_count(logits_f32: np.ndarray, s, sel_bias=None) -> int:
 
 # ------------------------------------------------------------------ backward bounds
 #
-# Element-wise bounds of the weight gradients. Every weight gradient is a sum of products
-# G[m, c] = sum_r A[r, m] * B[r, c] whose operands the GPU holds in bf16 (8 significant
-# bits: each rounding is off by at most 2^-8 of the value), each rounded once from a value
-# that is itself a rounded product chain, accumulated in fp32. Its error against the FP64
-# backward (given the same logits and routes) is bounded with every operand replaced by
-# the magnitude of its own chain:
-#   dy = bf16(w * dout)            |dy| <= |w| |dout|
-#   dh = dy . W2 (fp32)             mag(dh) = |dy| . |W2|
-#   dg = bf16(dh * u * silu'(g)),   mag(dg) = mag(dh) |u silu'(g)|,  mag(du) = mag(dh) |silu(g)|
-#   du = bf16(dh * silu(g))
-#   dW13 = [dg | du]^T . x          terms mag(dgu)[r, m] |x[r, c]|
-#   dW2  = dy^T . h, h = bf16(a)    terms |dy[r, m]| |a[r, c]|
-# (1) Worst case: two bf16 roundings on the chain (2 * 2^-8) plus fp32 accumulation over R
-#     rows (R * 2^-24, 1.2e-4 at R = 2000) stay below 2^-7 (1 + 2 %) of the linear sum
-#     S = sum_r |terms|: the bound 2^-6 S leaves a factor of two.
-# (2) Cancellation makes S loose where an expert has many rows (a wrong element of typical
-#     size can hide below it), so a second bound uses root-sum-squares Q = sqrt(sum_r
-#     t_r^2) of "typical" term sizes t_r, whose operands are the value itself plus the
-#     root-sum-square of the product that made it (e.g. typ(dh) = |dh| + sqrt(dy^2 .
-#     W2^2)): rounding errors of different terms are independent, each within 2^-7 of its
-#     typical size with a standard deviation below 2^-7 / sqrt(3), so the error sum has a
-#     standard deviation below 0.0046 Q; the bound 2^-3 Q is 27 of those, while an element
-#     taken from the wrong row or column is off by about Q.
-# The router's chain starts from the routing-weight gradient dw_j = dot32(dout, y): y is a
-# bf16 product of the bf16 h (its error <= 2^-7 of mag(y) = |h| . |W2|^T), so dw carries
-# 2^-7 of mag(dw) = |dout| . mag(y); the score and renormalisation steps carry it linearly
-# into mag(dlogits), which is rounded to bf16 once (2^-8) and contracted with x over T
-# tokens in fixed chunks (T * 2^-24): below 0.012 S at T = 4096, so the bound 2^-5 S; the
-# typical sizes follow the same chain (typ(y) = |y| + sqrt(h^2 . W2^2), typ(dw) = |dw| +
-# sqrt(dout^2 . typ(y)^2)) and the bound is 2^-2 Q (three roundings deep).
-WGRAD_EXPERT_C = 2.0 ** -6
+# Element-wise error bounds of the weight gradients against the FP64 backward (given the
+# same logits and routes). Every gradient element is a sum of products
+# G[m, c] = sum_r A[r, m] * B[r, c] whose operands the GPU computes in fp32 and holds in
+# bf16 (8 significant bits: a rounding is off by at most u = 2^-8 of the value), summed in
+# fp32 (n terms: at most g(n) = n * 2^-24 of the sum of their magnitudes). The bound follows
+# each operand's chain with first-order error propagation, in double:
+#   g, u = x . Wg, x . Wu (fp32 over H)     e_g = g(H) |x|.|Wg|,  e_u = g(H) |x|.|Wu|
+#   h = bf16(silu(g) u)                     e_h = u |h| + |u silu'(g)| e_g + |silu(g)| e_u
+#   y = bf16(h . W2^T) (fp32 over I)        e_y = (u + g(I)) |h|.|W2|^T + e_h.|W2|^T
+#   dw_j = dot32(dout, y)                   e_dw = |dout|.e_y + g(H) |dout|.|y|
+#   dy = bf16(w dout)                       e_dy = (u + 2^-20) |w dout|
+#   dh = dy . W2 (fp32 over H)              e_dh = (u + 2^-20 + g(H)) |dy|.|W2|   (= ... DH)
+#   dg = bf16(dh u silu'(g)),               e_dg = (u + ...) DH |u silu'| + DH (|silu'| e_u +
+#   du = bf16(dh silu(g))                          |u silu''| e_g), e_du likewise
+#   dW13 = [dg | du]^T . x, dW2 = dy^T . h, dW_router = bf16(dlogits)^T . x (fp32 over the
+#   rows, in fixed chunks for the router), dlogits carrying e_dw through the score and
+#   renormalisation steps linearly.
+# The test allows twice that bound (second-order terms). A bound of this worst-case kind is
+# loose where an expert has many rows and the terms cancel, so a wrong element of typical
+# size could hide below it; a second, statistical check uses root-sum-squares over the
+# rows, whose rounding errors are independent: Q = sqrt(sum_r t_r^2) of typical term sizes
+# t_r (each operand's value plus the root-sum-square of the product that made it), each
+# rounding within 2^-7 of its typical size with a standard deviation below 2^-7 / sqrt(3),
+# so the sum's standard deviation is below 0.0046 Q, and allowed 2^-3 Q (2^-2 Q for the
+# router, three roundings deep); plus 8 root-sum-squares of the rows' typical gate/up
+# errors (fp32 sums of H products, taken as 4 x 2^-24 sqrt(H) times their root-sum-square),
+# which cancellation in g or u makes large relative to h. An element taken from the wrong
+# row or column is off by about Q.
 WGRAD_EXPERT_CQ = 2.0 ** -3
-WGRAD_ROUTER_C = 2.0 ** -5
 WGRAD_ROUTER_CQ = 2.0 ** -2
+_U8 = 2.0 ** -8
+
+
+def _g(n):
+    return n * 2.0 ** -24
 
 
 def _sigma64(z):
     return 1.0 / (1.0 + np.exp(-z))
 
 
-def _lin_rss(a, b):
-    """(sum_r |a[r, m]| |b[r, c]|, sqrt(sum_r a[r, m]^2 b[r, c]^2)) for a, b >= 0."""
-    return a.T @ b, np.sqrt((a * a).T @ (b * b))
+def _silu_parts(g):
+    """silu(g), silu'(g), silu''(g) in double."""
+    s = _sigma64(g)
+    d1 = s * (1.0 + g * (1.0 - s))
+    d2 = s * (1.0 - s) * (2.0 + g * (1.0 - 2.0 * s))
+    return g * s, d1, d2
 
 
-def wgrad_scales64(dout, x, logits, w13, w2, ids, score_fn, renorm, route_scale, mask=None,
+def _rss(a, b):
+    return np.sqrt((a * a).T @ (b * b))
+
+
+def _expert_bounds(xr, dsgn_r, w_r, w13_e, w2_e, ad_r, shared):
+    """(bound13, bound2, Q13, Q2, G13, G2, e_dw, Y, typical e_dw) for one expert's rows:
+    error bounds, root-sum-squares of typical term sizes and of typical gate/up-induced
+    term errors, and the routing-weight gradient's error bound, magnitude and typical
+    gate/up-induced error per row."""
+    H = xr.shape[1]
+    I = w13_e.shape[0] // 2
+    R = xr.shape[0]
+    ax = np.abs(xr)
+    aw13 = np.abs(w13_e)
+    gu = xr @ w13_e.T
+    g, u = gu[:, :I], gu[:, I:]
+    mag = ax @ aw13.T
+    e_g, e_u = _g(H) * mag[:, :I], _g(H) * mag[:, I:]
+    rss = 4.0 * 2.0 ** -24 * np.sqrt(H) * np.sqrt((xr * xr) @ (w13_e * w13_e).T)
+    t_g, t_u = rss[:, :I], rss[:, I:]
+    sl, d1, d2 = _silu_parts(g)
+    a = sl * u
+    aa = np.abs(a)
+    gu_a = np.abs(u * d1) * e_g + np.abs(sl) * e_u        # g/u part of e_h
+    gu_a_t = np.abs(u * d1) * t_g + np.abs(sl) * t_u      # and its typical size
+    aw2 = np.abs(w2_e)
+    # rows of the forward's y: its magnitude and error (for the routing-weight gradient)
+    Y = aa @ aw2.T
+    e_y = (2 * _U8 + _g(I)) * Y + gu_a @ aw2.T
+    e_dw = np.einsum("nh,nh->n", ad_r, e_y) + _g(H) * np.einsum("nh,nh->n", ad_r, Y)
+    e_y_t = np.sqrt((gu_a_t * gu_a_t) @ (w2_e * w2_e).T)
+    e_dw_t = np.sqrt(np.einsum("nh,nh->n", ad_r ** 2, e_y_t ** 2))
+    # dy: exact for the shared expert (dy = dout), else one rounding of w dout
+    dy = (1.0 if shared else np.abs(w_r)[:, None]) * ad_r
+    r_dy = 0.0 if shared else _U8 + 2.0 ** -20
+    DH = dy @ aw2
+    f_g, f_u = np.abs(u * d1), np.abs(sl)
+    DGU = np.concatenate([DH * f_g, DH * f_u], axis=1)
+    gu_dgu = np.concatenate([DH * (np.abs(d1) * e_u + np.abs(u * d2) * e_g),
+                             DH * np.abs(d1) * e_g], axis=1)
+    e_dgu = (_U8 + r_dy + _g(H)) * DGU + gu_dgu
+    b13 = e_dgu.T @ ax + _g(R) * (DGU.T @ ax)
+    S2 = dy.T @ aa
+    b2 = (r_dy + _U8 + _g(R)) * S2 + dy.T @ gu_a
+    # typical sizes: the value plus the root-sum-square of the product that made it
+    sgn_dy = (1.0 if shared else w_r[:, None]) * dsgn_r
+    dht = np.abs(sgn_dy @ w2_e) + np.sqrt((dy * dy) @ (w2_e * w2_e))
+    t = np.concatenate([dht * f_g, dht * f_u], axis=1)
+    Q13 = _rss(t, ax)
+    Q2 = _rss(dy, aa)
+    tg = np.concatenate([dht * (np.abs(d1) * t_u + np.abs(u * d2) * t_g),
+                         dht * np.abs(d1) * t_g], axis=1)
+    G13 = _rss(tg, ax)
+    G2 = _rss(dy, gu_a_t)
+    return b13, b2, Q13, Q2, G13, G2, e_dw, Y, e_dw_t
+
+
+def wgrad_bounds64(dout, x, logits, w13, w2, ids, score_fn, renorm, route_scale, mask=None,
                    w13_s=None, w2_s=None, experts=()):
-    """Magnitude sums of the weight gradients' terms (see above), in double, for the given
-    logits and routes: {name: (S, Q)} for names "dw13[e]", "dw2[e]" (e in `experts`),
-    "dw_router" and, with a shared expert, "dw13_s", "dw2_s". w13/w2 are indexable per
-    expert (float64 arrays); the router's sums need every routed row."""
+    """Error bounds of the weight gradients (see above), in double, for the given logits
+    and routes: {name: (bound, Q, Qg)} (Qg: root-sum-square of the typical gate/up-induced
+    term errors) for "dw13[e]", "dw2[e]" (e in
+    `experts`), "dw_router" and, with a shared expert, "dw13_s", "dw2_s". w13/w2 are
+    indexable per expert (float64 arrays); the router's bound needs every routed row."""
     from oracle import backward64 as B
     x = np.asarray(x, np.float64)
     ids = np.asarray(ids, np.int64)
     T, H = x.shape
     K = ids.shape[1]
     kept = np.ones(T, bool) if mask is None else np.asarray(mask) != 0
-    ad = np.where(kept[:, None], np.abs(np.asarray(dout, np.float64)), 0.0)
+    dsgn = np.where(kept[:, None], np.asarray(dout, np.float64), 0.0)
+    ad = np.abs(dsgn)
     ax = np.abs(x)
     logits = np.asarray(logits, np.float64)
     s = B.scores64(logits, score_fn)
@@ -157,37 +220,32 @@ def wgrad_scales64(dout, x, logits, w13, w2, ids, score_fn, renorm, route_scale,
             w = np.where(D[:, None] != 0, sel / D[:, None], 0.0) * route_scale
     else:
         w = sel * route_scale
-    dwmag = np.zeros((T, K))     # linear magnitude of dw
-    dwtyp = np.zeros((T, K))     # typical size of dw
-    dsgn = np.where(kept[:, None], np.asarray(dout, np.float64), 0.0)
+    dwmag = np.zeros((T, K))     # |dout| . |y|: the routing-weight gradient's magnitude
+    dwerr = np.zeros((T, K))     # its error bound
+    dwtyp = np.zeros((T, K))     # its typical size
     res = {}
     for e in np.unique(ids[valid]):
         tt, jj = np.nonzero((ids == e) & kept[:, None])
         if tt.size == 0:
             continue
         w13_e, w2_e = np.asarray(w13[e], np.float64), np.asarray(w2[e], np.float64)
+        b13, b2, Q13, Q2, G13, G2, e_dw, Y, e_dw_t = _expert_bounds(
+            x[tt], dsgn[tt], w[tt, jj], w13_e, w2_e, ad[tt], False)
+        dwmag[tt, jj] = np.einsum("nh,nh->n", ad[tt], Y)
+        dwerr[tt, jj] = e_dw
         I = w13_e.shape[0] // 2
         gu = x[tt] @ w13_e.T
-        g, u = gu[:, :I], gu[:, I:]
-        sg = _sigma64(g)
-        a = g * sg * u
-        aa = np.abs(a)
-        aw2 = np.abs(w2_e)
-        dwmag[tt, jj] = np.einsum("nh,nh->n", ad[tt], aa @ aw2.T)
-        ytyp = np.abs(a @ w2_e.T) + np.sqrt((a * a) @ (w2_e * w2_e).T)
-        dwtyp[tt, jj] = (np.abs(np.einsum("nh,nh->n", dsgn[tt], a @ w2_e.T))
-                         + np.sqrt(np.einsum("nh,nh->n", ad[tt] ** 2, ytyp ** 2)))
+        a = _silu_parts(gu[:, :I])[0] * gu[:, I:]
+        yv = a @ w2_e.T
+        yt = np.abs(yv) + np.sqrt((a * a) @ (w2_e * w2_e).T)
+        dwtyp[tt, jj] = (np.abs(np.einsum("nh,nh->n", dsgn[tt], yv))
+                         + np.sqrt(np.einsum("nh,nh->n", ad[tt] ** 2, yt ** 2))
+                         + 2.0 ** 7 * e_dw_t)
         if int(e) in experts:
-            dy = np.abs(w[tt, jj])[:, None] * ad[tt]
-            dh = dy @ aw2
-            dht = np.abs((w[tt, jj][:, None] * dsgn[tt]) @ w2_e) + np.sqrt((dy * dy) @ (w2_e * w2_e))
-            fg, fu = np.abs(u * sg * (1.0 + g * (1.0 - sg))), np.abs(g * sg)
-            S13 = np.concatenate([dh * fg, dh * fu], axis=1).T @ ax[tt]
-            t = np.concatenate([dht * fg, dht * fu], axis=1)
-            Q13 = np.sqrt((t * t).T @ (ax[tt] * ax[tt]))
-            res[f"dw13[{int(e)}]"] = (S13, Q13)
-            res[f"dw2[{int(e)}]"] = (dy.T @ aa, np.sqrt((dy * dy).T @ (aa * aa)))
-    # router: magnitudes through the renormalisation and the score function
+            res[f"dw13[{int(e)}]"] = (b13, Q13, G13)
+            res[f"dw2[{int(e)}]"] = (b2, Q2, G2)
+
+    # router: magnitudes and errors through the renormalisation and the score function
     def dlogits_mag(dwm):
         if renorm:
             with np.errstate(divide="ignore", invalid="ignore"):
@@ -211,34 +269,27 @@ def wgrad_scales64(dout, x, logits, w13, w2, ids, score_fn, renorm, route_scale,
         dl[~kept] = 0.0
         return dl
 
-    dl_lin, dl_typ = dlogits_mag(dwmag), dlogits_mag(dwtyp)
-    res["dw_router"] = (dl_lin.T @ ax, np.sqrt((dl_typ * dl_typ).T @ (ax * ax)))
+    DL = dlogits_mag(dwmag)
+    e_dl = dlogits_mag(dwerr) + _U8 * DL
+    dl_typ = dlogits_mag(dwtyp)
+    res["dw_router"] = (e_dl.T @ ax + _g(T) * (DL.T @ ax), _rss(dl_typ, ax), 0.0)
     if w13_s is not None:
-        w13s, w2s = np.asarray(w13_s, np.float64), np.asarray(w2_s, np.float64)
-        Is = w13s.shape[0] // 2
-        gu = x @ w13s.T
-        g, u = gu[:, :Is], gu[:, Is:]
-        sg = _sigma64(g)
-        dh = ad @ np.abs(w2s)
-        dht = np.abs(dsgn @ w2s) + np.sqrt((ad * ad) @ (w2s * w2s))
-        fg, fu = np.abs(u * sg * (1.0 + g * (1.0 - sg))), np.abs(g * sg)
-        t = np.concatenate([dht * fg, dht * fu], axis=1)
-        res["dw13_s"] = (np.concatenate([dh * fg, dh * fu], axis=1).T @ ax,
-                         np.sqrt((t * t).T @ (ax * ax)))
-        aa = np.abs(g * sg * u)
-        res["dw2_s"] = (ad.T @ aa, np.sqrt((ad * ad).T @ (aa * aa)))
+        b13, b2, Q13, Q2, G13, G2, _, _, _ = _expert_bounds(
+            x, dsgn, None, np.asarray(w13_s, np.float64), np.asarray(w2_s, np.float64), ad, True)
+        res["dw13_s"] = (b13, Q13, G13)
+        res["dw2_s"] = (b2, Q2, G2)
     return res
 
 
-def assert_within_scales(gpu, ref, scales, c, cq, what):
-    """|gpu - ref| <= c * S and <= cq * Q element by element (S, Q = linear and
-    root-sum-square magnitude sums of the element's terms). Returns the largest fraction
-    of either bound used."""
+def assert_within_bounds(gpu, ref, bounds, cq, what):
+    """|gpu - ref| <= 2 * bound and <= cq * Q + 8 * Qg, element by element. Returns the
+    largest fraction of either allowance used."""
+    bound, Q, Qg = bounds
     g = np.asarray(gpu, np.float64)
     err = np.abs(g - ref)
     used = 0.0
-    for lim, name in ((c * scales[0] + 1e-30, f"{c:.3g} x linear sum"),
-                      (cq * scales[1] + 1e-30, f"{cq:.3g} x root-sum-square")):
+    for lim, name in ((2.0 * bound + 1e-30, "twice the error bound"),
+                      (cq * Q + 8.0 * Qg + 1e-30, f"{cq:.3g} x root-sum-square")):
         r = err / lim
         i = np.unravel_index(np.argmax(r), r.shape)
         if r[i] > 1.0:

@@ -42,7 +42,7 @@ def test_status_strings(lib):
     assert N.status_string(0) == "ok"
     for code in (-1, -2, -3, -4, -5, -6):
         assert N.status_string(code) != "unknown status"
-    assert lib.moe_abi_version() == 103
+    assert lib.moe_abi_version() == 104
 
 
 GOOD = dict(T=64, H=128, E=8, K=2, I=256)
@@ -226,3 +226,10 @@ def test_permute_noalloc_size_limit(lib):
         pytest.skip("the accepted edge would launch on the fake pointers")
     assert call(T=(2048 * 2048) // 8, E=128, K=8) == N.MOE_ERR_DEVICE
     assert call(T=1, E=1024, K=16) == N.MOE_ERR_DEVICE
+
+
+def test_pipeline_wait_selftest_rejects_bad_arguments(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.moe_pipeline_wait_selftest(None, 100000, None) == N.MOE_ERR_ARG
+    assert lib.moe_pipeline_wait_selftest(fake, 10, None) == N.MOE_ERR_ARG
+    assert lib.moe_pipeline_wait_selftest(fake, 3 * 10**9, None) == N.MOE_ERR_ARG

@@ -145,7 +145,8 @@ def test_route_golden_two_token(golden):
 
 
 @pytest.mark.parametrize("T,K,E", [(1, 1, 8), (64, 2, 8), (3001, 8, 128), (8192, 1, 8),
-                                   (2048, 6, 256), (777, 16, 1024), (20000, 8, 128)])
+                                   (2048, 6, 256), (777, 16, 1024), (20000, 8, 128),
+                                   (40000, 8, 256), (5000, 16, 1024)])
 def test_permute_bit_exact(T, K, E):
     rng = np.random.default_rng(T + K + E)
     # skewed expert choice (uneven loads, some experts empty), masked tokens, bad ids
@@ -176,8 +177,13 @@ def test_permute_bit_exact(T, K, E):
                                                   (1000, 8, 2048, False, True),
                                                   (333, 6, 4096, True, True),
                                                   (4096, 1, 4096, False, False),
-                                                  (100, 16, 256, True, False)])
+                                                  (100, 16, 256, True, False),
+                                                  (700, 16, 512, True, True),
+                                                  (2000, 3, 1024, True, False),
+                                                  (300, 4, 2176, False, True)])
 def test_combine_bit_exact(T, K, H, shared, masked):
+    """Rank-order combine, bit-exact against the oracle: every K width, a shared expert,
+    masks, skipped terms and hidden sizes that are and are not multiples of 256."""
     rng = np.random.default_rng(T * 7 + K)
     rows = T * K
     y = synthetic.normal_bf16(rows, H, 1.5, T + K, "x")
