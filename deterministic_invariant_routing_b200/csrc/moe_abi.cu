@@ -184,8 +184,8 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
     p.ldo = I;
     p.status = status;
     if (gather != nullptr) return launch_tc_gemm_pair(p, st);
-    // full 256-row tiles (and tails over 128 rows) on CTA pairs, short tails on single SMs
-    // (the same bits either way; about 0.5 % faster on the bench workload)
+    // experts of more than 128 rows on CTA pairs (the last tile padded), smaller ones on
+    // single SMs: no expert's weights are read by both kernels (the same bits either way)
     p.skip_tails = 1;
     const cudaError_t e = launch_tc_gemm_pair(p, st);
     if (e != cudaSuccess) return e;
@@ -211,8 +211,7 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     p.out = y;
     p.ldo = H;
     p.status = status;
-    // (the 1-SM tail kernel measured slower here: down's 12 k-block tiles do not amortise
-    // its extra operand bytes and partial last wave)
+    // (all tiles on CTA pairs: with short K the one-SM tiles measured no faster here)
     return launch_tc_gemm_pair(p, st);
 }
 

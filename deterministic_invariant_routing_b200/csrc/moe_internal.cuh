@@ -153,13 +153,13 @@ struct GemmProblem {
     int b_k_rows;            //   N contiguous), read without transposing (EPI_WGRAD: [k, n])
     int a_mn;                // EPI_WGRAD: A given MN-major, [k, a_rows] (features contiguous)
     int skip_tails;          // EPI_SWIGLU / EPI_BF16, K-major, no gather: the pair kernel leaves
-                             // each group's last rows to launch_tc_gemm_tail when at most 128
+                             // groups of at most 128 rows to launch_tc_gemm_tail
 };
 
 // the grouped expert products on CTA pairs
 cudaError_t launch_tc_gemm_pair(const GemmProblem& p, cudaStream_t st);
-// the rows a skip_tails pair launch left (each group's last n % 256 rows when 0 < n % 256
-// <= 128): one 128-row tile per such group on a single SM (tcgen05 cta_group::1, M = 128)
+// the groups a skip_tails pair launch left (those of 1..128 rows): one 128-row tile per
+// such group on a single SM (tcgen05 cta_group::1, M = 128)
 cudaError_t launch_tc_gemm_tail(const GemmProblem& p, cudaStream_t st);
 
 // the router product: logits[T,E] = x . Wr^T (+ logit_bias), fp32

@@ -45,10 +45,17 @@ __global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __rest
     __syncthreads();
     const int64_t base = (int64_t)blockIdx.x * kChunk;
     int bad = 0;
-    for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
-        const int64_t a = base + i;
-        if (a >= A) break;
-        const int e = ids[a];
+    // all of this thread's ids are loaded before any is counted (independent loads in flight)
+    constexpr int kPer = kChunk / (kWarps * 32);
+    int ev[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int64_t a = base + threadIdx.x + (int64_t)q * blockDim.x;
+        ev[q] = a < A ? ids[a] : -1;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int e = ev[q];
         if (e >= 0 && e < E) atomicAdd(&sh[e], 1);
         else if (e >= E) ++bad;
     }
@@ -66,8 +73,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts
     __shared__ int32_t warp_tot[32];
     const int e = threadIdx.x;
     int32_t total = 0;
-    if (e < E)
-        for (int b = 0; b < nblocks; ++b) total += counts[(int64_t)b * E + e];
+    // eight blocks' counts loaded at a time (independent loads in flight)
+    if (e < E) {
+        int b = 0;
+        for (; b + 8 <= nblocks; b += 8) {
+            int32_t c[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) c[q] = counts[(int64_t)(b + q) * E + e];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) total += c[q];
+        }
+        for (; b < nblocks; ++b) total += counts[(int64_t)b * E + e];
+    }
     // block-wide exclusive scan of total over e
     const int lane = e & 31, wid = e >> 5;
     int32_t incl = total;
@@ -93,7 +110,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = excl + total;
         int32_t run = excl;
-        for (int b = 0; b < nblocks; ++b) {
+        int b = 0;
+        for (; b + 8 <= nblocks; b += 8) {
+            int32_t c[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) c[q] = counts[(int64_t)(b + q) * E + e];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                counts[(int64_t)(b + q) * E + e] = run;
+                run += c[q];
+            }
+        }
+        for (; b < nblocks; ++b) {
             const int32_t c = counts[(int64_t)b * E + e];
             counts[(int64_t)b * E + e] = run;
             run += c;
@@ -116,11 +144,15 @@ __global__ void __launch_bounds__(kWarps * 32) place_kernel(const int32_t* __res
     for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wbase[i] = 0;
     __syncthreads();
     const int64_t wstart = (int64_t)blockIdx.x * kChunk + (int64_t)wid * kPerWarp;
+    // this lane's expert of every round, loaded once up front (independent loads in flight)
+    constexpr int kRounds = kPerWarp / 32;
+    int ev[kRounds];
+#pragma unroll
+    for (int q = 0; q < kRounds; ++q) ev[q] = expert_of(ids, wstart + 32 * q + lane, A, E);
     // pass 1: per-warp counts
-    for (int r = 0; r < kPerWarp; r += 32) {
-        const int e = expert_of(ids, wstart + r + lane, A, E);
-        if (e >= 0) atomicAdd(&wbase[wid * E + e], 1);
-    }
+#pragma unroll
+    for (int q = 0; q < kRounds; ++q)
+        if (ev[q] >= 0) atomicAdd(&wbase[wid * E + ev[q]], 1);
     __syncthreads();
     // per expert: scan over warps, seeded with the block's base row
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -135,9 +167,10 @@ __global__ void __launch_bounds__(kWarps * 32) place_kernel(const int32_t* __res
     // pass 2: ranks within each round of 32 from the peer masks, rounds in order
     const unsigned lt_mask = (1u << lane) - 1u;
     int32_t* my = wbase + wid * E;
-    for (int r = 0; r < kPerWarp; r += 32) {
-        const int64_t a = wstart + r + lane;
-        const int e = expert_of(ids, a, A, E);
+#pragma unroll
+    for (int q = 0; q < kRounds; ++q) {
+        const int64_t a = wstart + 32 * q + lane;
+        const int e = ev[q];
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         int32_t row = -1;
         if (e >= 0) row = my[e] + __popc(peers & lt_mask);

@@ -11,30 +11,37 @@
 namespace moe {
 namespace {
 
+// The constants of the contract's exp_rl and ln_rl, fixed at compile time: ln 2 rounded to
+// the nearest multiple of 2^-12 (12 significant bits, 2839 / 4096: n * head is exact for
+// |n| <= 127), the fp32 rounding of the remainder, fp32(log2 e), fp32(sqrt 2), and the
+// series coefficients 1/k! and 1/(2k+1), each the fp32 rounding (a constant-expression
+// cast rounds to nearest) of its double value.
+constexpr double kLn2d = 0.693147180559945309417232121458;
+constexpr float kLn2Head = (float)(2839.0 / 4096.0);
+constexpr float kLn2Tail = (float)(kLn2d - 2839.0 / 4096.0);
+constexpr float kLog2e = (float)1.442695040888963407359924681002;
+constexpr float kSqrt2 = (float)1.414213562373095048801688724;
+static_assert(2839.0 / 4096.0 - kLn2d < 1.0 / 8192.0 && kLn2d - 2839.0 / 4096.0 < 1.0 / 8192.0,
+              "2839/4096 is ln 2 to the nearest 2^-12");
+
 // exp_rl: Cody & Waite additive range reduction (x = n ln2 + r, ln2 split in a 12-bit
 // head whose products with n are exact and an fp32 tail), then the degree-7 Taylor
 // polynomial of e^r by Horner with fused multiply-adds, scaled by 2^n built from the
 // exponent field. Specials: NaN -> NaN, x < -87 -> +0, x > 88 -> +inf.
 __device__ __forceinline__ float exp_rl(float x)
 {
-    // ln 2 rounded to the nearest multiple of 2^-12 (12 significant bits: n * head is
-    // exact for |n| <= 127), and the fp32 rounding of the remainder.
-    const double kLn2 = 0.693147180559945309417232121458;
-    const float kHead = __double2float_rn(rint(kLn2 * 4096.0) / 4096.0);
-    const float kTail = __double2float_rn(kLn2 - (double)kHead);
-    const float kLog2e = __double2float_rn(1.442695040888963407359924681002);
     if (isnan(x)) return x;
     if (x < -87.0f) return 0.0f;
     if (x > 88.0f) return __int_as_float(0x7f800000);
     const float n = rintf(__fmul_rn(x, kLog2e));
-    float r = __fmaf_rn(-n, kHead, x);
-    r = __fmaf_rn(-n, kTail, r);
+    float r = __fmaf_rn(-n, kLn2Head, x);
+    r = __fmaf_rn(-n, kLn2Tail, r);
     // Taylor coefficients 1/k!, k = 7 .. 0, each rounded once to fp32
-    float p = __double2float_rn(1.0 / 5040.0);
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 720.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 120.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 24.0));
-    p = __fmaf_rn(p, r, __double2float_rn(1.0 / 6.0));
+    float p = (float)(1.0 / 5040.0);
+    p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
@@ -48,25 +55,22 @@ __device__ __forceinline__ float exp_rl(float x)
 // then k ln 2 added with the two-part ln 2 of exp_rl.
 __device__ __forceinline__ float ln_rl(float v)
 {
-    const double kLn2 = 0.693147180559945309417232121458;
-    const float kHead = __double2float_rn(rint(kLn2 * 4096.0) / 4096.0);
-    const float kTail = __double2float_rn(kLn2 - (double)kHead);
     const uint32_t b = __float_as_uint(v);
     int k = (int)(b >> 23) - 127;
     float m = __uint_as_float((b & 0x7fffffu) | 0x3f800000u);
-    if (m > __double2float_rn(1.414213562373095048801688724)) {
+    if (m > kSqrt2) {
         m = __fmul_rn(m, 0.5f);
         k += 1;
     }
     const float f = __fsub_rn(m, 1.0f);  // exact (Sterbenz)
     const float z = __fdiv_rn(f, __fadd_rn(2.0f, f));
     const float w = __fmul_rn(z, z);
-    float q = __fmaf_rn(w, __double2float_rn(1.0 / 9.0), __double2float_rn(1.0 / 7.0));
-    q = __fmaf_rn(w, q, __double2float_rn(1.0 / 5.0));
-    q = __fmaf_rn(w, q, __double2float_rn(1.0 / 3.0));
+    float q = __fmaf_rn(w, (float)(1.0 / 9.0), (float)(1.0 / 7.0));
+    q = __fmaf_rn(w, q, (float)(1.0 / 5.0));
+    q = __fmaf_rn(w, q, (float)(1.0 / 3.0));
     const float lnm = __fmaf_rn(__fmul_rn(2.0f, __fmul_rn(z, w)), q, __fmul_rn(2.0f, z));
     const float kf = __int2float_rn(k);
-    return __fmaf_rn(kf, kHead, __fmaf_rn(kf, kTail, lnm));
+    return __fmaf_rn(kf, kLn2Head, __fmaf_rn(kf, kLn2Tail, lnm));
 }
 
 // log1p_rl, u >= 0: Goldberg's formula u * ln(1 + u) / ((1 + u) - 1), u itself when

@@ -12,10 +12,7 @@ namespace {
 
 constexpr int BK = 64;                              // k-block: one 128-byte swizzle row
 constexpr long long kTimeoutCycles = 2000000000LL;  // about a second at B200 clocks
-#ifndef MOE_SMEM_BUDGET
-#define MOE_SMEM_BUDGET 196608
-#endif
-constexpr int kSmemBudget = MOE_SMEM_BUDGET;        // bytes for the operand ring
+constexpr int kSmemBudget = 196608;                 // bytes for the operand ring
 
 // ------------------------------------------------------------------ PTX wrappers
 

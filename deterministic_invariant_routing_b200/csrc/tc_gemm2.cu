@@ -70,8 +70,7 @@ struct PairArgs {
                                  // value (gradient) in a row
     const float* bias;           // EPI_F32: per-column bias or NULL
     int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
-    int skip_tails;              // leave each group's last rows to the 1-SM tail kernel when
-                                 // they fit one CTA (at most 128 past the last full tile)
+    int skip_tails;              // leave groups of at most 128 rows to the 1-SM tail kernel
 };
 
 template <int EPI, int NP>
@@ -246,8 +245,9 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
         const int per = (G + 31) / 32;
         const int beg = lane * per < G ? lane * per : G;
         const int end = beg + per < G ? beg + per : G;
+        // with skip_tails, groups of at most 128 rows are the one-SM tail kernel's
         auto tiles_of = [&](int n) -> int {
-            return args.skip_tails ? n / PM + (n % PM > HM ? 1 : 0) : (n + PM - 1) / PM;
+            return (args.skip_tails && n <= HM) ? 0 : (n + PM - 1) / PM;
         };
         int sum = 0;
         for (int g = beg; g < end; ++g) {
@@ -290,14 +290,16 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
             uint32_t phase = 0;
             uint32_t armed = 0, armed_phase = 0;
             const uint32_t fb0 = mapa_shared(full_bar(0), 0);  // the leader's full[0]
+            // this CTA's B rows of a tile
+            auto b_row_of = [&](const PairTile& tt) -> int {
+                return kGateUp ? tt.g * args.b_rows_per_group + (leader ? 0 : args.half_rows) +
+                                     tt.n * kBRows
+                               : tt.g * args.b_rows_per_group + tt.n * NP + (int)rank * kBRows;
+            };
             for (int t = cluster; t < total && !*abort_flag; t += nclusters) {
                 const PairTile ti = decode(t);
                 const int arow = (int)ti.row0 + (int)rank * HM;
-                const int brow = kGateUp ? ti.g * args.b_rows_per_group +
-                                               (leader ? 0 : args.half_rows) + ti.n * kBRows
-                                 : kWgrad ? ti.n * NP + (int)rank * kBRows
-                                          : ti.g * args.b_rows_per_group + ti.n * NP +
-                                                (int)rank * kBRows;
+                const int brow = kWgrad ? ti.n * NP + (int)rank * kBRows : b_row_of(ti);
                 bool ok = true;
                 for (int kb = 0; kb < ti.kbs; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status)) {

@@ -1,9 +1,11 @@
 // The short last tiles of the grouped expert products on single SMs.
 //
-// A CTA-pair tile is 256 rows; a group (expert) whose row count leaves 1..128 rows past its
-// last full tile would fill only one CTA of a pair, so the pair kernel (tc_gemm2.cu, run with
-// skip_tails) leaves those rows here: one 128-row tile per such group and N tile, on one SM
-// with tcgen05.mma cta_group::1 (M = 128, N = 256, K = 16 per instruction). The operands,
+// A CTA-pair tile is 256 rows; a group (expert) of at most 128 rows would fill only one CTA
+// of a pair, so the pair kernel (tc_gemm2.cu, run with skip_tails) leaves such groups here:
+// one 128-row tile per group and N tile, on one SM with tcgen05.mma cta_group::1 (M = 128,
+// N = 256, K = 16 per instruction). Larger groups stay whole on the pairs, their last tile
+// padded: a group split between the two kernels would have its weights read from memory by
+// each of them. The operands,
 // the k-block order (64 wide, increasing, four K=16 steps each), the fp32 accumulation in
 // TMEM and the epilogue arithmetic are the pair kernel's, so a row gets the same bits
 // whichever kernel computes it (the batch-sweep and gather-path tests check this).
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
         auto row_off = [&](int g) -> int {
             return args.offsets ? args.offsets[g] : (g == 0 ? 0 : args.rows);
         };
-        auto has_tail = [&](int n) -> int { return (n % 256 > 0 && n % 256 <= TM) ? 1 : 0; };
+        auto has_tail = [&](int n) -> int { return (n > 0 && n <= TM) ? 1 : 0; };
         const int per = (G + 31) / 32;
         const int beg = lane * per < G ? lane * per : G;
         const int end = beg + per < G ? beg + per : G;
@@ -136,8 +138,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
             else hi = mid - 1;
         }
         ti.g = lo;
-        const int n_rows = toffs[lo + 1] - toffs[lo];
-        ti.row0 = (int64_t)toffs[lo] + (n_rows / 256) * 256;
+        ti.row0 = (int64_t)toffs[lo];  // the whole group (at most 128 rows)
         ti.row_end = toffs[lo + 1];
         return ti;
     };
@@ -147,16 +148,19 @@ __global__ void __launch_bounds__(kTailThreads, 1)
             // ---------------------------------------------------------- TMA producer
             int stage = 0;
             uint32_t phase = 0, armed = 0, armed_phase = 0;
+            auto b_rows = [&](const TailTile& tt, int& r0, int& r1) {
+                if (EPI == EPI_SWIGLU) {
+                    r0 = tt.g * args.b_rows_per_group + tt.n * 128;
+                    r1 = r0 + args.half_rows;
+                } else {
+                    r0 = tt.g * args.b_rows_per_group + tt.n * TN;
+                    r1 = r0 + 128;
+                }
+            };
             for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
                 const TailTile ti = decode(t);
                 int b0, b1;  // the two 128-row B boxes of the N tile
-                if (EPI == EPI_SWIGLU) {
-                    b0 = ti.g * args.b_rows_per_group + ti.n * 128;
-                    b1 = b0 + args.half_rows;
-                } else {
-                    b0 = ti.g * args.b_rows_per_group + ti.n * TN;
-                    b1 = b0 + 128;
-                }
+                b_rows(ti, b0, b1);
                 bool ok = true;
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.status)) {
