@@ -81,18 +81,22 @@ def source_sha(rels):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key, rows):
-    """DRAM bytes (read + write) per launch of a kernel at `rows` routed rows, from a
-    committed ncu summary (profiles/ncu_traffic.json): single-launch captures at two sizes
-    of the same layer give fixed bytes (weights) plus bytes per routed row, evaluated at
-    `rows`. None when the kernel's sources changed since the counters were taken."""
+def ncu_traffic(kernel_key, rows, workload=None):
+    """DRAM bytes (read + write) per launch of a kernel, from a committed ncu summary
+    (profiles/ncu_traffic.json): the single-launch capture of this workload when there is
+    one, else the straight line through the captures at two smaller sizes of the same layer
+    (fixed bytes of the weights plus bytes per routed row) at `rows`. None when the kernel's
+    sources changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
         if rec["source_sha"] != source_sha(rec["sources"]):
             return None
-        return rec["fixed_bytes"] + rec["bytes_per_row"] * rows
+        cap = rec.get("captures", {}).get(workload)
+        if cap is not None and cap["routed_rows"] == rows:
+            return cap["bytes"]
+        return round(rec["fixed_bytes"] + rec["bytes_per_row"] * rows)
     except Exception:
         return None
 
@@ -601,7 +605,7 @@ def main():
         "roofline": {"bound": bound, "kernel": "gate_up grouped GEMM + SwiGLU (tcgen05)",
                      "achieved": achieved, "peak": pk_k, "unit": unit,
                      "frac": achieved / pk_k, **fracs,
-                     "traffic": ncu_traffic("gate_up", rows),
+                     "traffic": ncu_traffic("gate_up", rows, f"{s.name}_T{s.T}"),
                      "peak_source": pk_desc, "peak_regime": regime,
                      "regime_rule": "burst when the timed steps plus the stage-split pass "
                                     f"keep the GPU busy under 1 s (here {busy_ms:.0f} ms)",

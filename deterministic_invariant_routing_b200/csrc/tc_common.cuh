@@ -366,15 +366,15 @@ __host__ __device__ constexpr uint32_t make_idesc_major(int m, int n, bool a_mn,
     return make_idesc(m, n) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
-// bf16 round-to-nearest-even of two floats packed low/high (NaN stays NaN, quieted)
+// bf16 round-to-nearest-even of two floats packed low/high
 __device__ __forceinline__ uint32_t bf16x2_rne(float lo, float hi)
 {
-    auto cvt = [](float f) -> uint32_t {
-        uint32_t u = __float_as_uint(f);
-        if ((u & 0x7fffffffu) > 0x7f800000u) return (u >> 16) | 0x40u;
-        return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
-    };
-    return cvt(lo) | (cvt(hi) << 16);
+    // one conversion instruction for the pair (round to nearest even; a NaN becomes the
+    // canonical bf16 NaN): far cheaper in the epilogues than the integer rounding formula,
+    // whose shifts and selects made down's epilogue ALU-bound
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
