@@ -43,7 +43,7 @@ def parse():
     p.add_argument("--workload", default="qwen3_30b_a3b")
     p.add_argument("--T", type=int, default=16384)
     p.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
-    p.add_argument("--e2e-chunk", type=int, default=5120,
+    p.add_argument("--e2e-chunk", type=int, default=6144,
                    help="tokens per chunk of the host-memory call (copies overlap compute)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
@@ -146,6 +146,11 @@ class ClockSampler:
                 else nv.nvmlDeviceGetHandleByIndex(int(self.gpu_id))
             self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
             self.thread.start()
+            # the first reading before the timed region starts, so that a region of a few
+            # milliseconds is still sampled
+            t0 = time.perf_counter()
+            while not self.samples and time.perf_counter() - t0 < 0.5:
+                time.sleep(0.0005)
             self.source = f"NVML every {self.period_s * 1e3:.0f} ms"
             return self
         except Exception:
@@ -183,6 +188,7 @@ class ClockSampler:
                                               if v.lower() == "active"}))
 
     def summary(self):
+        # samples from the start of the timed region on (plus the one reading just before it)
         sm = [a for a, _, _ in self.samples]
         mx = max((b for _, b, _ in self.samples), default=0.0)
         reasons = set()

@@ -397,7 +397,7 @@ def forward_host_workspace_bytes(cfg: Config, chunk: int) -> int:
 
 
 def forward_host(cfg: Config, x_host, w_router, w13, w2, logit_bias=None, sel_bias=None,
-                 token_mask=None, w13_s=None, w2_s=None, out_host=None, chunk: int = 5120,
+                 token_mask=None, w13_s=None, w2_s=None, out_host=None, chunk: int = 6144,
                  ws=None, status=None, check: bool = True):
     """The layer from and to host memory in one C-ABI call, transfers overlapped with the
     compute in chunks around `chunk` tokens (half-size first and last chunks, middle ones of
@@ -444,7 +444,7 @@ class MoELayer:
         self.ws = _ws(workspace_bytes(cfg.with_T(self.max_T), N.MOE_STAGE_FORWARD), dev, None)
         self.status = new_status(dev)
 
-    def forward_host(self, x_host, out_host=None, chunk: int = 5120, token_mask=None,
+    def forward_host(self, x_host, out_host=None, chunk: int = 6144, token_mask=None,
                      check=True):
         """The layer from pinned host memory to pinned host memory (see forward_host)."""
         T = x_host.shape[0]
