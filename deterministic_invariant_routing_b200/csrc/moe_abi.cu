@@ -10,6 +10,12 @@
 
 namespace moe {
 
+// SMs left to the one-SM kernel of small experts when it runs beside the pair kernel:
+// below 192 routed rows per expert on average, and from 192 to 511 (measured against
+// 24/48 and 48/80 on the 30B-A3B and sigmoid layers)
+constexpr int kSideSmsLow = 64;
+constexpr int kSideSmsHigh = 36;
+
 int num_sms()
 {
     static int cached[64] = {};
@@ -185,8 +191,16 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
     p.status = status;
     if (gather != nullptr) return launch_tc_gemm_pair(p, st);
     // experts of more than 128 rows on CTA pairs (the last tile padded), smaller ones on
-    // single SMs: no expert's weights are read by both kernels (the same bits either way)
+    // single SMs: no expert's weights are read by both kernels (the same bits either way).
+    // Where small experts are common (about 64 to 512 rows per expert on average) the two
+    // launches run side by side: the pair tiles keep the tensor pipes busy while the small
+    // experts' tiles, bound by reading their weights, use the SMs left to them. Which SMs
+    // run which tiles changes nothing in any row's arithmetic.
     p.skip_tails = 1;
+    const int64_t per_expert = groups > 0 ? grouped_rows / groups : 0;
+    p.side_sms = (per_expert >= 64 && per_expert < 192) ? kSideSmsLow
+                 : (per_expert >= 192 && per_expert < 512) ? kSideSmsHigh
+                                                            : 0;
     const cudaError_t e = launch_tc_gemm_pair(p, st);
     if (e != cudaSuccess) return e;
     return launch_tc_gemm_tail(p, st);
@@ -211,7 +225,17 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     p.out = y;
     p.ldo = H;
     p.status = status;
-    // (all tiles on CTA pairs: with short K the one-SM tiles measured no faster here)
+    // Where small experts are common, as for gate_up: their tiles on single SMs side by
+    // side with the pair tiles (run one after the other, the one-SM tiles measured no
+    // faster here: down's 12-k-block tiles are short).
+    const int64_t per_expert = groups > 0 ? a_rows / groups : 0;
+    if (offsets != nullptr && H % 256 == 0 && per_expert >= 64 && per_expert < 512) {
+        p.skip_tails = 1;
+        p.side_sms = per_expert < 192 ? kSideSmsLow : kSideSmsHigh;
+        const cudaError_t e = launch_tc_gemm_pair(p, st);
+        if (e != cudaSuccess) return e;
+        return launch_tc_gemm_tail(p, st);
+    }
     return launch_tc_gemm_pair(p, st);
 }
 

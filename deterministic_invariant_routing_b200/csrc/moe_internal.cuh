@@ -154,6 +154,10 @@ struct GemmProblem {
     int a_mn;                // EPI_WGRAD: A given MN-major, [k, a_rows] (features contiguous)
     int skip_tails;          // EPI_SWIGLU / EPI_BF16, K-major, no gather: the pair kernel leaves
                              // groups of at most 128 rows to launch_tc_gemm_tail
+    int side_sms;            // with skip_tails: > 0 runs the two launches side by side -- the
+                             // pair kernel on 148 - side_sms SMs signalling its dependents at
+                             // once, the one-SM kernel on side_sms SMs, waiting for the pair
+                             // kernel only before it exits; 0 runs them one after the other
 };
 
 // the grouped expert products on CTA pairs

@@ -71,6 +71,7 @@ struct PairArgs {
     const float* bias;           // EPI_F32: per-column bias or NULL
     int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
     int skip_tails;              // leave groups of at most 128 rows to the 1-SM tail kernel
+    int early_trigger;           // let the next kernel start on the SMs this launch leaves free
 };
 
 template <int EPI, int NP>
@@ -226,6 +227,9 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     }
     if (warp == 1) tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
     pdl_wait();  // the previous kernel's writes (offsets, operands) are visible from here on
+    // the one-SM kernel for small groups may run beside this one from now on (it reads
+    // nothing this launch writes, and waits for this launch before it exits)
+    if (args.early_trigger && threadIdx.x == 0) pdl_trigger();
     if (warp == 2 && EPI == EPI_WGRAD) {
         // groups by descending K length (ties: lower group first): order[rank] = group
         int32_t* kl = offs;
@@ -864,6 +868,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.bias = p.bias;
     a.b_k_rows = wgrad ? 0 : p.b_k_rows;
     a.skip_tails = p.skip_tails;
+    a.early_trigger = (p.skip_tails && p.side_sms > 0) ? 1 : 0;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;
@@ -873,6 +878,11 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     const int64_t max_tiles = wgrad ? (int64_t)groups * a.m_tiles * a.n_tiles
                                     : ((rows_total + PM - 1) / PM + groups) * a.n_tiles;
     int64_t clusters = max_clusters[dev];
+    if (a.early_trigger) {
+        // leave side_sms SMs to the one-SM kernel that runs beside this launch
+        const int64_t keep = (num_sms() - p.side_sms) / 2;
+        if (keep >= 1 && keep < clusters) clusters = keep;
+    }
     if (max_tiles < clusters) clusters = max_tiles;
     if (clusters < 1) clusters = 1;
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);

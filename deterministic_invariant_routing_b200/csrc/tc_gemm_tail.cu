@@ -42,6 +42,7 @@ struct TailArgs {
     void* out;
     int64_t ldo;
     int32_t* status;
+    int side;  // running beside the pair kernel: no wait at the start, a wait before exiting
 };
 
 struct TailTile {
@@ -93,7 +94,11 @@ __global__ void __launch_bounds__(kTailThreads, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) tmem_alloc(smem_u32(misc), 2 * TN);
-    pdl_wait();  // the previous kernel's writes (offsets, operands) are visible from here on
+    // The previous kernel's writes (offsets, operands) are visible from here on. Beside the
+    // pair kernel, that kernel is the pair launch, which started this one only after its own
+    // wait (so the dispatch that wrote offsets and operands has completed); this launch then
+    // waits for the pair launch before exiting, so the next kernel finds both complete.
+    if (!args.side) pdl_wait();
     if (warp == 2) {
         // groups with 1..128 rows past their last full 256-row tile, as a prefix count
         auto row_off = [&](int g) -> int {
@@ -320,6 +325,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (args.side) pdl_wait();  // the pair launch beside this one has completed
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -361,8 +367,10 @@ cudaError_t launch_tail_variant(const GemmProblem& p, cudaStream_t st)
     a.out = p.out;
     a.ldo = p.ldo;
     a.status = p.status;
-    // at most one tail tile per group and N tile
+    a.side = p.side_sms > 0 ? 1 : 0;
+    // at most one tail tile per group and N tile; beside the pair kernel, its side SMs
     int64_t grid = (int64_t)groups * a.n_tiles;
+    if (a.side && grid > p.side_sms) grid = p.side_sms;
     if (grid > num_sms()) grid = num_sms();
     if (grid < 1) grid = 1;
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kTailThreads), smem, st, ma, mb, mo, a);
