@@ -39,11 +39,11 @@ __device__ __forceinline__ int warp_argmax_id(unsigned long long k)
 
 // descending sort of a lane's keys: the optimal 5-exchange network for 4, odd-even
 // transposition otherwise (the order of equal keys cannot matter: keys are distinct)
-template <int NE>
-__device__ __forceinline__ void sort_desc(unsigned long long (&key)[NE])
+template <int NE, typename Key>
+__device__ __forceinline__ void sort_desc(Key (&key)[NE])
 {
     auto cx = [&](int a, int b) {
-        const unsigned long long ka = key[a], kb = key[b];
+        const Key ka = key[a], kb = key[b];
         const bool swap = ka < kb;
         key[a] = swap ? kb : ka;
         key[b] = swap ? ka : kb;
@@ -63,10 +63,49 @@ __device__ __forceinline__ void sort_desc(unsigned long long (&key)[NE])
     }
 }
 
-// NE = experts held per lane (E <= 32 * NE)
-// up to 128 experts the kernel fits 40 registers (6 resident blocks of 8 warps per SM):
-// its K selection rounds are a chain of warp reductions, so latency is hidden by warps
-template <int NE>
+// Selection of the K best keys of a warp whose lanes hold NE keys each, sorted descending
+// in every lane: K rounds of a warp arg-max over the lanes' heads, the winner dropping its
+// head. Lane j (j < K) returns the key of round j; for 32-bit keys *boundary receives the
+// best key left over.
+template <int NE, int KT, typename Key>
+__device__ __forceinline__ Key select_rounds(Key (&key)[NE], int K, int lane, Key* boundary)
+{
+    Key mine = 0;
+#pragma unroll
+    for (int j = 0; j < (KT > 0 ? KT : K); ++j) {
+        Key m;
+        if constexpr (sizeof(Key) == 8) {
+            const uint32_t hi = (uint32_t)(key[0] >> 32), lo = (uint32_t)key[0];
+            const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+            const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+            m = ((Key)mhi << 32) | mlo;
+        } else {
+            m = __reduce_max_sync(0xffffffffu, key[0]);
+        }
+        if (key[0] == m) {
+#pragma unroll
+            for (int i = 0; i + 1 < NE; ++i) key[i] = key[i + 1];
+            key[NE - 1] = 0;
+        }
+        if (lane == j) mine = m;
+    }
+    if constexpr (sizeof(Key) == 4)
+        if (boundary != nullptr) *boundary = __reduce_max_sync(0xffffffffu, key[0]);
+    return mine;
+}
+
+// NE = experts held per lane (E <= 32 * NE); KT = K when fixed at compile time, else 0.
+//
+// Selection. The exact key of expert e is the 64-bit (ordered choice bits, inverted id).
+// The common path selects on 32-bit keys that keep the top 32 - B choice bits and put the
+// inverted id in the low B bits (2^B > 32 NE, so every real key is nonzero): one reduction
+// per round instead of two, and half the data to sort and shift. Cutting choice bits keeps
+// the order of any two keys whose kept bits differ; the cut selection equals the exact one
+// when the kept bits of the picks in rank order, followed by the best key left over, are
+// strictly decreasing -- then each pick beats everything after it on the kept bits alone.
+// A token where two neighbours of that sequence share their kept bits (near-ties, equal
+// scores, NaN rows) is selected again on the exact 64-bit keys. Both paths give the same ids.
+template <int NE, int KT>
 __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const float* __restrict__ logits, int T, int E,
                                                     int K, const float* __restrict__ sel_bias,
                                                     const uint8_t* __restrict__ mask, int score_fn,
@@ -75,7 +114,11 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
                                                     int32_t* __restrict__ ids,
                                                     float* __restrict__ w, int32_t* status)
 {
+    constexpr int kIdBits = NE <= 1 ? 6 : NE <= 2 ? 7 : NE <= 4 ? 8 : NE <= 8 ? 9 : NE <= 16 ? 10 : 11;
+    constexpr uint32_t kIdMask = (1u << kIdBits) - 1u;  // > every id (ids < 32 NE)
+    static_assert((1 << kIdBits) > 32 * NE, "cut keys need room for every id");
     pdl_wait();
+    if (KT > 0) K = KT;
     extern __shared__ float choice_smem[];  // [warps][E], group-limited selection only
     const int lane = threadIdx.x & 31;
     float* cw = choice_smem + (threadIdx.x >> 5) * E;
@@ -92,25 +135,31 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
         }
         float s[NE];
         contract_scores<NE>(logits + (int64_t)t * E, E, score_fn, lane, s);
-        // selection keys; empty slots get key 0 (below every real key)
-        unsigned long long key[NE];
+        // choice values (empty slots are never keyed) and the cut keys
+        auto choice = [&](int i) -> float {
+            const int e = lane + 32 * i;
+            return sel_bias != nullptr ? __fadd_rn(s[i], sel_bias[e]) : s[i];
+        };
+        uint32_t ck[NE];
         bool any_nan = false;
 #pragma unroll
         for (int i = 0; i < NE; ++i) {
             const int e = lane + 32 * i;
             if (e < E) {
-                const float c = (sel_bias != nullptr) ? __fadd_rn(s[i], sel_bias[e]) : s[i];
+                const float c = choice(i);
                 any_nan |= isnan(c);
-                key[i] = select_key(c, e);
+                ck[i] = (order_bits(c) & ~kIdMask) | (kIdMask - (uint32_t)e);
                 if (n_group > 1) cw[e] = c;
             } else {
-                key[i] = 0ull;
+                ck[i] = 0u;
             }
         }
         if (__any_sync(0xffffffffu, any_nan)) nan_tokens += (lane == 0);
+        uint32_t kept = 0xffffffffu;  // group-limited selection: the kept groups
+        int gs = 1;
         if (n_group > 1) {
             __syncwarp();
-            const int gs = E / n_group;
+            gs = E / n_group;
             unsigned long long gk = 0ull;
             if (lane < n_group) {
                 unsigned long long k1 = 0ull, k2 = 0ull;
@@ -124,7 +173,7 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
                 gk = select_key(gs > 1 ? __fadd_rn(c1, c2) : c1, lane);
             }
             __syncwarp();  // the scan is done before the next token overwrites cw
-            uint32_t kept = 0u;
+            kept = 0u;
             for (int r = 0; r < topk_group; ++r) {
                 const int g = warp_argmax_id(gk);
                 kept |= 1u << g;
@@ -133,22 +182,30 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
 #pragma unroll
             for (int i = 0; i < NE; ++i) {
                 const int e = lane + 32 * i;
-                if (e < E && ((kept >> (e / gs)) & 1u) == 0u) key[i] = 0ull;
+                if (e < E && ((kept >> (e / gs)) & 1u) == 0u) ck[i] = 0u;
             }
         }
-        // each lane orders its own keys (descending) once; then K rounds of a warp arg-max
-        // over the lanes' heads, the winning lane dropping its head. Lane j keeps the id
-        // of round j; the scores stay where the lanes computed them and are fetched once.
-        sort_desc<NE>(key);
-        int my_id = -1;
-        for (int j = 0; j < K; ++j) {
-            const int e = warp_argmax_id(key[0]);
-            if (lane == (e & 31)) {
+        // cut-key selection, then the strict-decrease test of the kept bits (lane j holds
+        // the key of round j; the best key left over is the boundary)
+        sort_desc<NE>(ck);
+        uint32_t bnd;
+        const uint32_t mk = select_rounds<NE, KT>(ck, K, lane, &bnd);
+        const uint32_t top = mk & ~kIdMask;
+        const uint32_t nxt_lane = __shfl_down_sync(0xffffffffu, top, 1);
+        const uint32_t nxt = (lane == K - 1) ? (bnd & ~kIdMask) : nxt_lane;
+        int my_id = (int)(kIdMask - (mk & kIdMask));
+        if (__any_sync(0xffffffffu, lane < K && top == nxt)) {
+            // exact selection on the 64-bit keys
+            unsigned long long key[NE];
 #pragma unroll
-                for (int i = 0; i + 1 < NE; ++i) key[i] = key[i + 1];
-                key[NE - 1] = 0ull;
+            for (int i = 0; i < NE; ++i) {
+                const int e = lane + 32 * i;
+                const bool live = e < E && (n_group <= 1 || ((kept >> (e / gs)) & 1u) != 0u);
+                key[i] = live ? select_key(choice(i), e) : 0ull;
             }
-            if (lane == j) my_id = e;
+            sort_desc<NE>(key);
+            const unsigned long long m = select_rounds<NE, KT>(key, K, lane, static_cast<unsigned long long*>(nullptr));
+            my_id = (int)(0xffffffffu - (uint32_t)m);
         }
         // the unbiased score of this lane's pick: slot my_id / 32 of lane my_id % 32
         float my_s = 0.0f;
@@ -162,7 +219,9 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
         }
         // renormalisation denominator: the picks' scores added in rank order
         float den = __shfl_sync(0xffffffffu, my_s, 0);
-        for (int j = 1; j < K; ++j) den = __fadd_rn(den, __shfl_sync(0xffffffffu, my_s, j));
+#pragma unroll
+        for (int j = 1; j < (KT > 0 ? KT : K); ++j)
+            den = __fadd_rn(den, __shfl_sync(0xffffffffu, my_s, j));
         if (renorm && den == 0.0f) zero_den += (lane == 0);
         if (lane < K) {
             float wv;
@@ -180,8 +239,8 @@ __global__ void __launch_bounds__(256, (NE <= 4 ? 6 : 1)) route_kernel(const flo
     }
 }
 
-template <int NE>
-cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bias,
+template <int NE, int KT>
+cudaError_t launch_nk(const moe_cfg& c, const float* logits, const float* sel_bias,
                       const uint8_t* mask, int32_t* ids, float* w, int32_t* status,
                       cudaStream_t st)
 {
@@ -190,11 +249,27 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bi
     const int n_group = c.n_group > 1 ? c.n_group : 0;
     const size_t smem = n_group ? (size_t)wpb * c.E * sizeof(float) : 0;
     // one wave of resident blocks, each warp taking every (grid warps)-th token
-    const int cap = resident_blocks((const void*)route_kernel<NE>, threads, smem);
+    const int cap = resident_blocks((const void*)route_kernel<NE, KT>, threads, smem);
     if (blocks > cap) blocks = cap;
-    return launch_pdl(route_kernel<NE>, dim3(blocks), dim3(threads), smem, st, logits, c.T, c.E,
-                      c.K, sel_bias, mask, c.score_fn, c.renorm, c.route_scale, n_group,
+    return launch_pdl(route_kernel<NE, KT>, dim3(blocks), dim3(threads), smem, st, logits, c.T,
+                      c.E, c.K, sel_bias, mask, c.score_fn, c.renorm, c.route_scale, n_group,
                       c.topk_group, ids, w, status);
+}
+
+// the top-k sizes of the layers this library is built for get unrolled selection rounds
+template <int NE>
+cudaError_t launch_ne(const moe_cfg& c, const float* logits, const float* sel_bias,
+                      const uint8_t* mask, int32_t* ids, float* w, int32_t* status,
+                      cudaStream_t st)
+{
+    switch (c.K) {
+    case 1: return launch_nk<NE, 1>(c, logits, sel_bias, mask, ids, w, status, st);
+    case 2: return launch_nk<NE, 2>(c, logits, sel_bias, mask, ids, w, status, st);
+    case 4: return launch_nk<NE, 4>(c, logits, sel_bias, mask, ids, w, status, st);
+    case 6: return launch_nk<NE, 6>(c, logits, sel_bias, mask, ids, w, status, st);
+    case 8: return launch_nk<NE, 8>(c, logits, sel_bias, mask, ids, w, status, st);
+    default: return launch_nk<NE, 0>(c, logits, sel_bias, mask, ids, w, status, st);
+    }
 }
 
 }  // namespace

@@ -249,6 +249,51 @@ def test_route_injected_near_ties_bit_exact(name, T, n_near):
     assert n >= n_near // 2
 
 
+def _ulps_below(v, n):
+    """The float32 n representable steps below v (towards -inf), for finite v."""
+    u = int(np.array([v], np.float32).view(np.uint32)[0])
+    if u & 0x80000000:
+        u = min(u + n, 0xff7fffff)
+    elif u >= n:
+        u -= n
+    else:
+        u = 0x80000000 | (n - u)
+    return np.array([u], np.uint32).view(np.float32)[0]
+
+
+@pytest.mark.parametrize("name,T", [("qwen3_30b_a3b", 4096), ("dsv_sigmoid", 4096),
+                                    ("dspark", 2048)])
+def test_route_close_choices_every_rank_bit_exact(name, T):
+    """Pairs of choices a few ulps apart at every rank and at the K-th/(K+1)-th boundary:
+    for each token one expert's logit is set 2^k ulps below the logit of the expert picked
+    at rank r (k = 0 .. 12, r = 0 .. K), so their choices land in the same or in
+    neighbouring buckets of any fixed number of leading bits. The selection must still
+    match the oracle's exact order."""
+    s = synthetic.shape(name, T=T)
+    E, K = s.E, s.K
+    l = synthetic.random_logits(T, E, seed=s.seed + 70, std=2.0).numpy().astype(np.float32)
+    bias = None
+    if s.sel_bias_range is not None:
+        bias = synthetic.uniform_f32(E, s.sel_bias_range, s.seed, "sel_bias").numpy()
+        bias[1::2] = bias[0::2]
+    ids0, _, _ = oracle.route_fp32(l, min(K + 1, E), s.score_fn, s.renorm, s.route_scale,
+                                   sel_bias=bias)
+    for t in range(T):
+        r = t % min(K + 1, E)
+        a = int(ids0[t, r])
+        b = a ^ 1
+        if b >= E:
+            continue
+        k = (t // (K + 1)) % 13
+        l[t, b] = _ulps_below(l[t, a], 1 << k)
+    cfg = moe.Config.of(s)
+    _, ids, w = moe.route(cfg, logits=torch.from_numpy(l).to(DEV),
+                          sel_bias=None if bias is None else torch.from_numpy(bias).to(DEV))
+    r_ids, r_w, _ = oracle.route_fp32(l, K, s.score_fn, s.renorm, s.route_scale, sel_bias=bias)
+    assert np.array_equal(ids.cpu().numpy(), r_ids), np.argwhere(ids.cpu().numpy() != r_ids)[:5]
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), r_w.view(np.uint32))
+
+
 @pytest.mark.parametrize("name,T,keep", [("qwen3_30b_a3b", 4096, None), ("qwen3_30b_a3b", 3001, 0.8),
                                          ("dsv_sigmoid", 2048, 0.9), ("tiny", 64, None),
                                          ("dspark", 1000, 0.5), ("dsv_sqrtsoftplus", 2048, 0.9)])
