@@ -22,7 +22,9 @@ __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 // bf16 round-to-nearest-even of two floats packed low/high; a NaN keeps its sign and
-// payload's top bits and is made quiet (the contract's single downcast)
+// payload's top bits and is made quiet (the contract's single downcast). Without a NaN the
+// hardware conversion gives the same bits as the integer rounding below (round to nearest
+// even, overflow to infinity, subnormals kept) in one instruction per pair.
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
     auto cvt = [](float f) -> uint32_t {
@@ -30,7 +32,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
         if ((u & 0x7fffffffu) > 0x7f800000u) return (u >> 16) | 0x40u;
         return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
     };
-    return cvt(a) | (cvt(b) << 16);
+    if (isnan(a) || isnan(b)) return cvt(a) | (cvt(b) << 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
 }
 
 // VPT consecutive 16-byte vectors of one token per thread: the token's K row indices and

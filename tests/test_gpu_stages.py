@@ -203,6 +203,49 @@ def test_combine_bit_exact(T, K, H, shared, masked):
     assert np.array_equal(bits(out), ref)
 
 
+def test_combine_special_values_bit_exact():
+    """The combine's single bf16 downcast on values that exercise its rounding: infinities
+    (and inf - inf = NaN), sums that overflow only after rounding, fp32 subnormal results,
+    bf16 rounding ties (fp32 low halves of exactly 0x8000, odd and even) and signed zeros.
+    Finite and infinite outputs must match the oracle bit for bit, NaN outputs be NaN."""
+    T, K, H = 257, 8, 256
+    rng = np.random.default_rng(91)
+    rows = T * K
+    yb = synthetic.normal_bf16(rows, H, 1.0, 91, "x").view(torch.int16).numpy().view(np.uint16).copy()
+    w = rng.uniform(0, 1, (T, K)).astype(np.float32)
+    dest = rng.permutation(rows).astype(np.int32).reshape(T, K)
+    bf = lambda v: np.array([v], np.float32).view(np.uint32)[0] >> 16
+    # token rows of y by rank: plant specials in the first columns of a few tokens
+    for t in range(0, T, 5):
+        r = dest[t]
+        yb[r[0], 0] = bf(np.inf)
+        yb[r[1], 1] = bf(-np.inf)
+        yb[r[0], 2] = bf(np.inf)
+        yb[r[1], 2] = bf(-np.inf)                       # inf - inf: NaN
+        yb[r[:], 3] = 0x7f7f                            # largest bf16: the sum overflows
+        w[t, :] = np.maximum(w[t, :], 0.5)
+        yb[r[:], 4] = 0x0001                            # bf16 subnormals: fp32 subnormal sums
+        yb[r[:], 5] = 0x8000                            # -0
+        yb[r[2], 6] = 0x3f81                            # 1 + 2^-7: products near bf16 ties
+    for t in range(1, T, 7):                            # exact bf16 ties: 1 + 2^-8 (even
+        w[t, :] = 0.0                                   # down) and 1 + 2^-7 + 2^-8 (odd up)
+        w[t, 0] = np.float32(1.0 + 2.0 ** -8) if t % 2 else np.float32(1.0 + 2.0 ** -7 + 2.0 ** -8)
+        yb[dest[t][0], 7] = 0x3f80
+    cfg = moe.Config(T=T, H=H, E=8, K=K, I=128)
+    y = torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16)
+    out = moe.combine(cfg, y.to(DEV), torch.from_numpy(w).to(DEV), torch.from_numpy(dest).to(DEV))
+    ref = oracle.combine_fp32(y, w, dest)
+    g = bits(out)
+    nan_ref = ((ref & 0x7f80) == 0x7f80) & ((ref & 0x7f) != 0)
+    nan_g = ((g & 0x7f80) == 0x7f80) & ((g & 0x7f) != 0)
+    assert np.array_equal(nan_g, nan_ref)
+    assert nan_ref.any()
+    assert np.array_equal(g[~nan_ref], ref[~nan_ref])
+    assert ((ref[~nan_ref] & 0x7fff) == 0x7f80).any()        # infinities among them
+    assert ((ref[~nan_ref] & 0x7f80) == 0).any()             # and subnormals or zeros
+    assert set(ref[1::7, 7].tolist()) == {0x3f80, 0x3f82}    # both ties, rounded to even
+
+
 def test_combine_cancellation_order(golden):
     c = golden("tree_sum_and_combine_order.json")["combine_case"]
     K, H = c["K"], 128
