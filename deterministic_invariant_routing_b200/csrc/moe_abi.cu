@@ -931,8 +931,8 @@ MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w
     if (cfg->T == 0) return MOE_OK;
     if ((rc = check_device()) != MOE_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((rc = rec(stage_events, 0, st)) != MOE_OK) return rc;
     if ((rc = cuda_rc(cudaMemsetAsync(status, 0, MOE_STATUS_WORDS * 4, st))) != MOE_OK) return rc;
+    if ((rc = rec(stage_events, 0, st)) != MOE_OK) return rc;  // the router stage starts here
     return forward_impl(*cfg, x, w_router, logit_bias, sel_bias, token_mask, w13, w2, w13_s, w2_s,
                         out, logits, topk_ids, topk_w, offsets, status, ws, stage_events, st);
 }

@@ -273,9 +273,10 @@ MOE_API int moe_combine_invariant(const moe_cfg* cfg, const uint16_t* y, const f
  *  status     int32[MOE_STATUS_WORDS] device, required.
  *  ws         moe_workspace_bytes(cfg, MOE_STAGE_FORWARD) bytes.
  *  stage_events NULL, or MOE_NUM_STAGE_EVENTS cudaEvent_t handles recorded on `stream`
- *             at the stage boundaries: [0] start, [1] after router logits, [2] after
- *             routing, [3] after dispatch, [4] after gate_up, [5] after down, [6] after
- *             the shared expert, [7] after the combine (timing only).
+ *             at the stage boundaries: [0] start (after the status words are cleared),
+ *             [1] after router logits, [2] after routing, [3] after dispatch, [4] after
+ *             gate_up, [5] after down, [6] after the shared expert, [7] after the combine
+ *             (timing only).
  */
 MOE_API int moe_forward(const moe_cfg* cfg, const uint16_t* x, const uint16_t* w_router,
                         const float* logit_bias, const float* sel_bias,
