@@ -10,11 +10,13 @@
 
 namespace moe {
 
-// SMs left to the one-SM kernel of small experts when it runs beside the pair kernel:
-// below 192 routed rows per expert on average, and from 192 to 511 (measured against
-// 24/48 and 48/80 on the 30B-A3B and sigmoid layers)
-constexpr int kSideSmsLow = 64;
-constexpr int kSideSmsHigh = 36;
+// SMs the one-SM kernel of small experts starts on beside the pair kernel: below 192
+// routed rows per expert on average, and from 192 to 511. It takes its tiles from a
+// counter, so its CTAs past these take the small experts left when pair CTAs finish;
+// measured against 64/36 and 32/16 on the 30B-A3B layer (T = 2048 .. 16384) and the
+// sigmoid layer (T = 4096, 8192): 48/24 was the fastest or within 1 % everywhere.
+constexpr int kSideSmsLow = 48;
+constexpr int kSideSmsHigh = 24;
 
 int num_sms()
 {
@@ -88,9 +90,10 @@ int check_device()
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// scratch of moe_grouped_ffn: h [T*K, I] (+ h_shared [T, I_shared]), bf16
+// scratch of moe_grouped_ffn: h [T*K, I] (+ h_shared [T, I_shared]), bf16, and the tile
+// counters of the two one-SM launches (gate_up's, down's)
 struct FfnLayout {
-    size_t h, h_s, total;
+    size_t h, h_s, ctr, total;
 };
 
 FfnLayout ffn_layout(const moe_cfg& c)
@@ -102,6 +105,8 @@ FfnLayout ffn_layout(const moe_cfg& c)
     off += up(A * c.I * 2);
     L.h_s = off;
     off += up((size_t)c.T * c.I_shared * 2);
+    L.ctr = off;
+    off += up(2 * sizeof(int32_t));
     L.total = off;
     return L;
 }
@@ -169,9 +174,10 @@ int router_and_route(const moe_cfg& c, const uint16_t* x, const uint16_t* wr,
 // gate_up + SwiGLU over grouped rows: h[r] = silu(a_r . W1g^T) * (a_r . W1u^T), where
 // a_r is row gather[r] of a when gather is given (the dispatch fused into the GEMM's
 // operand loads) and row r otherwise
+// (tail_ctr: a device int for the one-SM launch's tile counter, or NULL)
 cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, int64_t grouped_rows,
                     const int32_t* offsets, int groups, int rows, const uint16_t* w13, int H, int I,
-                    uint16_t* h, int32_t* status, cudaStream_t st)
+                    uint16_t* h, int32_t* status, int32_t* tail_ctr, cudaStream_t st)
 {
     GemmProblem p{};
     p.epilogue = EPI_SWIGLU;
@@ -197,6 +203,7 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
     // experts' tiles, bound by reading their weights, use the SMs left to them. Which SMs
     // run which tiles changes nothing in any row's arithmetic.
     p.skip_tails = 1;
+    p.tail_ctr = tail_ctr;
     const int64_t per_expert = groups > 0 ? grouped_rows / groups : 0;
     p.side_sms = (per_expert >= 64 && per_expert < 192) ? kSideSmsLow
                  : (per_expert >= 192 && per_expert < 512) ? kSideSmsHigh
@@ -208,7 +215,8 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
 
 // down over grouped rows: y[r] = h_r . W2^T
 cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int groups, int rows,
-                 const uint16_t* w2, int H, int I, uint16_t* y, int32_t* status, cudaStream_t st)
+                 const uint16_t* w2, int H, int I, uint16_t* y, int32_t* status, int32_t* tail_ctr,
+                 cudaStream_t st)
 {
     GemmProblem p{};
     p.epilogue = EPI_BF16;
@@ -231,6 +239,7 @@ cudaError_t down(const uint16_t* h, int64_t a_rows, const int32_t* offsets, int 
     const int64_t per_expert = groups > 0 ? a_rows / groups : 0;
     if (offsets != nullptr && H % 256 == 0 && per_expert >= 64 && per_expert < 512) {
         p.skip_tails = 1;
+        p.tail_ctr = tail_ctr;
         p.side_sms = per_expert < 192 ? kSideSmsLow : kSideSmsHigh;
         const cudaError_t e = launch_tc_gemm_pair(p, st);
         if (e != cudaSuccess) return e;
@@ -330,22 +339,24 @@ int ffn_impl(const moe_cfg& c, const uint16_t* x, const uint16_t* x_perm,
     const FfnLayout L = ffn_layout(c);
     const int64_t A = (int64_t)c.T * c.K;
     uint16_t* h = at<uint16_t>(ws, L.h);
+    int32_t* ctr = at<int32_t>(ws, L.ctr);
     int rc = x_perm != nullptr
                  ? cuda_rc(gate_up(x_perm, A, nullptr, A, offsets, c.E, 0, w13, c.H, c.I, h, status,
-                                   st))
+                                   ctr, st))
                  : cuda_rc(gate_up(x, c.T, perm_token, A, offsets, c.E, 0, w13, c.H, c.I, h, status,
-                                   st));
+                                   nullptr, st));
     if (rc != MOE_OK) return rc;
     if ((rc = rec(ev, 4, st)) != MOE_OK) return rc;
-    rc = cuda_rc(down(h, A, offsets, c.E, 0, w2, c.H, c.I, y, status, st));
+    rc = cuda_rc(down(h, A, offsets, c.E, 0, w2, c.H, c.I, y, status, ctr + 1, st));
     if (rc != MOE_OK) return rc;
     if ((rc = rec(ev, 5, st)) != MOE_OK) return rc;
     if (c.I_shared > 0 && w13_s != nullptr) {
         uint16_t* h_s = at<uint16_t>(ws, L.h_s);
         rc = cuda_rc(gate_up(x, c.T, nullptr, c.T, nullptr, 1, c.T, w13_s, c.H, c.I_shared, h_s,
-                             status, st));
+                             status, nullptr, st));
         if (rc != MOE_OK) return rc;
-        rc = cuda_rc(down(h_s, c.T, nullptr, 1, c.T, w2_s, c.H, c.I_shared, y_shared, status, st));
+        rc = cuda_rc(down(h_s, c.T, nullptr, 1, c.T, w2_s, c.H, c.I_shared, y_shared, status,
+                          nullptr, st));
         if (rc != MOE_OK) return rc;
     }
     return rec(ev, 6, st);
@@ -643,7 +654,7 @@ int train_intermediates(const moe_cfg& c, const uint16_t* x, const int32_t* ids,
     MOE_TRY(launch_zero_pad_rows(x_perm, H, offsets, poff, E, st));
     MOE_TRY(launch_gather_rows(c, x, dest_pad, x_perm, st));
     MOE_TRY(gate_up_save(x_perm, rp, poff, E, 0, w13, H, I, h, at<float>(ws, L.gu), status, st));
-    MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, at<uint16_t>(ws, L.y), status, st));
+    MOE_TRY(down(h, rp, poff, E, 0, w2, H, I, at<uint16_t>(ws, L.y), status, nullptr, st));
     if (Is > 0)
         MOE_TRY(gate_up_save(x, T, nullptr, 1, T, w13s, H, Is, at<uint16_t>(ws, L.h_s),
                              at<float>(ws, L.gu_s), status, st));
@@ -1104,7 +1115,7 @@ MOE_API int moe_forward_train(const moe_cfg* cfg, const uint16_t* x, const uint1
     if (c.I_shared > 0) {
         y_s = at<uint16_t>(ws, L.y_s);
         if ((rc = cuda_rc(down(at<uint16_t>(ws, L.h_s), c.T, nullptr, 1, c.T, w2_s, c.H,
-                               c.I_shared, y_s, status, st))) != MOE_OK)
+                               c.I_shared, y_s, status, nullptr, st))) != MOE_OK)
             return rc;
     }
     return cuda_rc(launch_combine(c, at<uint16_t>(ws, L.y), topk_w, at<int32_t>(ws, L.dest_pad),

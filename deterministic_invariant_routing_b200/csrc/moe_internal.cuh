@@ -154,6 +154,8 @@ struct GemmProblem {
     int a_mn;                // EPI_WGRAD: A given MN-major, [k, a_rows] (features contiguous)
     int skip_tails;          // EPI_SWIGLU / EPI_BF16, K-major, no gather: the pair kernel leaves
                              // groups of at most 128 rows to launch_tc_gemm_tail
+    int32_t* tail_ctr;       // with skip_tails: a device int the pair launch zeroes and the
+                             // one-SM launch deals its tiles from, or NULL (dealt by CTA index)
     int side_sms;            // with skip_tails: > 0 runs the two launches side by side -- the
                              // pair kernel on 148 - side_sms SMs signalling its dependents at
                              // once, the one-SM kernel on side_sms SMs, waiting for the pair

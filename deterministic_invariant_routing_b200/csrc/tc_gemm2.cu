@@ -72,6 +72,7 @@ struct PairArgs {
     int b_k_rows;                // MN-major B: K rows of each group (0: one shared B)
     int skip_tails;              // leave groups of at most 128 rows to the 1-SM tail kernel
     int early_trigger;           // let the next kernel start on the SMs this launch leaves free
+    int32_t* tail_ctr;           // the one-SM launch's tile counter, zeroed here, or NULL
 };
 
 template <int EPI, int NP>
@@ -227,6 +228,12 @@ __global__ void __launch_bounds__(Cfg2<EPI, NP>::kThreads, 1)
     }
     if (warp == 1) tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
     pdl_wait();  // the previous kernel's writes (offsets, operands) are visible from here on
+    // the one-SM kernel's tile counter starts at zero: written and fenced before this CTA's
+    // trigger, and the one-SM launch starts only once every CTA of this one has triggered
+    if (args.tail_ctr != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        *args.tail_ctr = 0;
+        __threadfence();
+    }
     // the one-SM kernel for small groups may run beside this one from now on (it reads
     // nothing this launch writes, and waits for this launch before it exits)
     if (args.early_trigger && threadIdx.x == 0) pdl_trigger();
@@ -869,6 +876,7 @@ cudaError_t launch_pair_variant(const GemmProblem& p, cudaStream_t st)
     a.b_k_rows = wgrad ? 0 : p.b_k_rows;
     a.skip_tails = p.skip_tails;
     a.early_trigger = (p.skip_tails && p.side_sms > 0) ? 1 : 0;
+    a.tail_ctr = p.skip_tails ? p.tail_ctr : nullptr;
     a.gather_rows = p.gather_rows;
     a.a = p.a;
     a.k = p.k;

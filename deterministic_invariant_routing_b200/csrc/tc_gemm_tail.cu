@@ -30,6 +30,8 @@ constexpr uint32_t kTB = TN * BK * 2;        // 32 KiB
 constexpr uint32_t kTStage = kTA + kTB;      // 48 KiB
 constexpr int kTStages = kSmemBudget / (int)kTStage;  // 4
 constexpr uint32_t kTEpi = 4 * 2 * 2048;     // 4 warps x 2 store tiles of 32 x 32 bf16
+constexpr int kTQ = 4;                       // tile-index queue from the producer to the others
+constexpr int kTBars = 2 * kTStages + 5 + 2 * kTQ;
 
 struct TailArgs {
     int k_blocks;
@@ -43,6 +45,8 @@ struct TailArgs {
     int64_t ldo;
     int32_t* status;
     int side;  // running beside the pair kernel: no wait at the start, a wait before exiting
+    int32_t* tile_ctr;  // tiles taken from this counter (zeroed by the pair launch), or NULL:
+                        // tile t on CTA t mod grid
 };
 
 struct TailTile {
@@ -71,9 +75,12 @@ __global__ void __launch_bounds__(kTailThreads, 1)
     auto tfull_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (uint32_t)(2 * S + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (uint32_t)(2 * S + 4);
-    uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);  // [0] tmem, [1] abort
+    auto qfull_bar = [&](int q) { return bar0 + 8u * (uint32_t)(2 * S + 5 + q); };
+    auto qempty_bar = [&](int q) { return bar0 + 8u * (uint32_t)(2 * S + 5 + kTQ + q); };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(bars + kTBars);  // [0] tmem, [1] abort
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-    int32_t* tprefix = reinterpret_cast<int32_t*>(misc + 4);  // [groups + 1] tail tiles before g
+    volatile int32_t* tq = reinterpret_cast<volatile int32_t*>(misc + 4);  // [kTQ] tile indices
+    int32_t* tprefix = reinterpret_cast<int32_t*>(misc + 8);  // [groups + 1] tail tiles before g
     int32_t* toffs = tprefix + (args.groups + 1);            // [groups + 1] row offsets
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -89,6 +96,10 @@ __global__ void __launch_bounds__(kTailThreads, 1)
             mbar_init(tempty_bar(a), 4 * 32);
         }
         mbar_init(drain_bar, 1);
+        for (int q = 0; q < kTQ; ++q) {
+            mbar_init(qfull_bar(q), 1);
+            mbar_init(qempty_bar(q), 1 + 4);  // the MMA thread and the four epilogue warps
+        }
         misc[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -162,7 +173,25 @@ __global__ void __launch_bounds__(kTailThreads, 1)
                     r1 = r0 + 128;
                 }
             };
-            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+            // every tile index goes through the queue (-1 ends it), taken from the counter
+            // when there is one, else this CTA's share t = blockIdx.x + k gridDim.x
+            int qi = 0, next = blockIdx.x;
+            uint32_t qphase = 0;
+            for (;;) {
+                int t = -1;
+                if (!*abort_flag) {
+                    t = args.tile_ctr ? atomicAdd(args.tile_ctr, 1) : next;
+                    next += gridDim.x;
+                    if (t >= total) t = -1;
+                }
+                if (!wait_bounded(qempty_bar(qi), qphase ^ 1u, abort_flag, args.status)) break;
+                tq[qi] = t;
+                mbar_arrive(qfull_bar(qi));
+                if (++qi == kTQ) {
+                    qi = 0;
+                    qphase ^= 1u;
+                }
+                if (t < 0) break;
                 const TailTile ti = decode(t);
                 int b0, b1;  // the two 128-row B boxes of the N tile
                 b_rows(ti, b0, b1);
@@ -187,7 +216,9 @@ __global__ void __launch_bounds__(kTailThreads, 1)
                 }
                 if (!ok) break;
             }
-            pdl_trigger();
+            // beside the pair kernel the next launch is scheduled when this one completes:
+            // started earlier, its CTAs could hold SMs that this launch's later CTAs need
+            if (!args.side) pdl_trigger();
             if (*abort_flag) {
                 for (int s = 0; s < S; ++s)
                     if (armed & (1u << s))
@@ -202,8 +233,17 @@ __global__ void __launch_bounds__(kTailThreads, 1)
             const uint64_t bd0 = sw128_desc(sB0);
             int stage = 0;
             uint32_t phase = 0;
-            int i = 0;
-            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x, ++i) {
+            int qi = 0;
+            uint32_t qphase = 0;
+            for (int i = 0;; ++i) {
+                if (!wait_bounded(qfull_bar(qi), qphase, abort_flag, args.status)) break;
+                const int t = tq[qi];
+                mbar_arrive(qempty_bar(qi));
+                if (++qi == kTQ) {
+                    qi = 0;
+                    qphase ^= 1u;
+                }
+                if (t < 0 || *abort_flag) break;
                 const int acc = i & 1;
                 if (!wait_bounded(tempty_bar(acc), (((uint32_t)i >> 1) & 1u) ^ 1u, abort_flag,
                                   args.status))
@@ -269,8 +309,20 @@ __global__ void __launch_bounds__(kTailThreads, 1)
                     dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
         };
-        int i = 0;
-        for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x, ++i) {
+        int qi = 0;
+        uint32_t qphase = 0;
+        for (int i = 0;; ++i) {
+            int t = -1;
+            if (lane == 0 && wait_bounded(qfull_bar(qi), qphase, abort_flag, args.status)) {
+                t = tq[qi];
+                mbar_arrive(qempty_bar(qi));
+            }
+            t = __shfl_sync(0xffffffffu, t, 0);
+            if (++qi == kTQ) {
+                qi = 0;
+                qphase ^= 1u;
+            }
+            if (t < 0 || *abort_flag) break;
             const TailTile ti = decode(t);
             const int acc = i & 1;
             int ok = 1;
@@ -338,7 +390,7 @@ cudaError_t launch_tail_variant(const GemmProblem& p, cudaStream_t st)
 {
     auto kernel = tc_gemm_tail_kernel<EPI>;
     const int groups = p.offsets ? p.groups : 1;
-    const size_t smem = 1024 + (size_t)kTStages * kTStage + kTEpi + (2 * kTStages + 5) * 8 + 16 +
+    const size_t smem = 1024 + (size_t)kTStages * kTStage + kTEpi + kTBars * 8 + 32 +
                         (size_t)2 * (groups + 1) * sizeof(int32_t);
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -368,9 +420,12 @@ cudaError_t launch_tail_variant(const GemmProblem& p, cudaStream_t st)
     a.ldo = p.ldo;
     a.status = p.status;
     a.side = p.side_sms > 0 ? 1 : 0;
-    // at most one tail tile per group and N tile; beside the pair kernel, its side SMs
+    a.tile_ctr = p.tail_ctr;
+    // at most one tail tile per group and N tile. Beside the pair kernel with tiles dealt by
+    // CTA index: its side SMs. With the counter: a CTA per SM, the first side_sms of them
+    // running beside the pair tiles and the rest taking what is left as pair CTAs finish.
     int64_t grid = (int64_t)groups * a.n_tiles;
-    if (a.side && grid > p.side_sms) grid = p.side_sms;
+    if (a.side && a.tile_ctr == nullptr && grid > p.side_sms) grid = p.side_sms;
     if (grid > num_sms()) grid = num_sms();
     if (grid < 1) grid = 1;
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kTailThreads), smem, st, ma, mb, mo, a);
