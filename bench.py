@@ -81,17 +81,20 @@ def source_sha(rels):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key, rows, workload=None):
+def ncu_traffic(kernel_key, rows, layer, workload=None):
     """DRAM bytes (read + write) per launch of a kernel, from a committed ncu summary
     (profiles/ncu_traffic.json): the single-launch capture of this workload when there is
     one, else the straight line through the captures at two smaller sizes of the same layer
-    (fixed bytes of the weights plus bytes per routed row) at `rows`. None when the kernel's
-    sources changed since the counters were taken."""
+    (fixed bytes of the weights plus bytes per routed row) at `rows`. None for a layer the
+    record does not cover, or when the kernel's sources changed since the counters were
+    taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
         if rec["source_sha"] != source_sha(rec["sources"]):
+            return None
+        if rec.get("layer") != layer:
             return None
         cap = rec.get("captures", {}).get(workload)
         if cap is not None and cap["routed_rows"] == rows:
@@ -611,7 +614,7 @@ def main():
         "roofline": {"bound": bound, "kernel": "gate_up grouped GEMM + SwiGLU (tcgen05)",
                      "achieved": achieved, "peak": pk_k, "unit": unit,
                      "frac": achieved / pk_k, **fracs,
-                     "traffic": ncu_traffic("gate_up", rows, f"{s.name}_T{s.T}"),
+                     "traffic": ncu_traffic("gate_up", rows, s.name, f"{s.name}_T{s.T}"),
                      "peak_source": pk_desc, "peak_regime": regime,
                      "regime_rule": "burst when the timed steps plus the stage-split pass "
                                     f"keep the GPU busy under 1 s (here {busy_ms:.0f} ms)",
