@@ -240,3 +240,34 @@ def test_tied_router_rows_pick_lower_id():
     ob = bits(r["out"])
     for a, b in ((0, 1), (10, 11), (20, 30), (40, 63)):
         assert np.array_equal(ids[a], ids[b]) and np.array_equal(ob[a], ob[b])
+
+
+@pytest.mark.parametrize("E,H,T", [(33, 128, 300), (100, 2048, 1000), (300, 1024, 257),
+                                   (1024, 8192, 130), (8, 4096, 513), (256, 4096, 129)])
+def test_router_logits_odd_shapes(E, H, T):
+    """The router product at expert counts and hidden sizes the layer shapes do not reach:
+    column tiles of 64, 128 and 256 experts with part of the last one past E, one or several
+    column tiles, K split over clusters of 1, 2 and 8 CTAs (and the CTA-pair path at
+    E = 256), ragged last row tiles. Every token's logits against the FP64 product within
+    the same bound as the layer tests; the logit bias added after the K reduction."""
+    rng = np.random.default_rng(E * 7 + H)
+    x = synthetic.normal_bf16(T, H, 1.0, E + H, "x")
+    wr = synthetic.normal_bf16(E, H, 0.02, E + H, "w_router")
+    lb = torch.from_numpy(rng.normal(0, 0.5, E).astype(np.float32))
+    cfg = moe.Config(T=T, H=H, E=E, K=1, I=128)
+    logits, _, _ = moe.route(cfg, x=x.to(DEV), w_router=wr.to(DEV), logit_bias=lb.to(DEV),
+                             check=False)
+    torch.cuda.synchronize()
+    g = logits.cpu().numpy()
+    ref = oracle.logits64(x, wr, lb)
+    xf = x.float().numpy().astype(np.float64)
+    scale = np.abs(xf) @ np.abs(wr.float().numpy().astype(np.float64)).T
+    assert g.shape == (T, E)
+    assert np.all(np.abs(g - ref) <= 2e-5 * scale + 1e-6)
+    # the same tokens in another batch give the same bits (the split depends on H only)
+    sub = x[T // 3:T // 3 + 5].clone()
+    cfg5 = moe.Config(T=5, H=H, E=E, K=1, I=128)
+    l5, _, _ = moe.route(cfg5, x=sub.to(DEV), w_router=wr.to(DEV), logit_bias=lb.to(DEV),
+                         check=False)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(l5), bits(logits[T // 3:T // 3 + 5]))
