@@ -396,3 +396,60 @@ def test_combine_invariant_bit_exact_and_order_free(T, K, H, shared, masked, spr
     out2 = moe.combine(cfg, dev(y), dev(w2), dev(d2), y_shared=dev(ys), token_mask=dev(mask),
                        order_invariant=True)
     assert np.array_equal(bits(out2), bits(out))
+
+
+def _special_bf16(rng, shape):
+    """bf16 bits: normals of every exponent, with zeros of both signs, subnormals, infinities
+    and NaN mixed in."""
+    n = int(np.prod(shape))
+    sign = rng.integers(0, 2, n).astype(np.uint16) << 15
+    expo = rng.integers(100, 150, n).astype(np.uint16)
+    kind = rng.random(n)
+    expo[kind < 0.06] = rng.integers(1, 12, int((kind < 0.06).sum()))       # tiny normals
+    expo[(kind >= 0.06) & (kind < 0.12)] = rng.integers(200, 255, int(((kind >= 0.06) & (kind < 0.12)).sum()))
+    mant = rng.integers(0, 128, n).astype(np.uint16)
+    b = sign | (expo << 7) | mant
+    b[(kind >= 0.12) & (kind < 0.17)] = sign[(kind >= 0.12) & (kind < 0.17)]            # +-0
+    sub = (kind >= 0.17) & (kind < 0.22)
+    b[sub] = sign[sub] | rng.integers(1, 128, int(sub.sum())).astype(np.uint16)          # subnormal
+    b[(kind >= 0.22) & (kind < 0.225)] = 0x7f80
+    b[(kind >= 0.225) & (kind < 0.23)] = 0xff80
+    b[(kind >= 0.23) & (kind < 0.235)] = 0x7fc0
+    return b.reshape(shape)
+
+
+@pytest.mark.parametrize("T,K,H,shared", [(300, 8, 256, True), (200, 6, 512, False), (64, 16, 128, True)])
+def test_combine_invariant_special_values(T, K, H, shared):
+    """The order-invariant combine on terms of every kind -- zeros of both signs, bf16
+    subnormals, normals from the bottom to the top of the exponent range, infinities, NaN,
+    and weights that are zero, subnormal, negative, huge or infinite -- matches the oracle
+    bit for bit wherever the oracle's result is a number (NaN wherever it is NaN), and
+    permuting each token's terms changes no bit."""
+    rng = np.random.default_rng(T + 7 * K)
+    rows = T * K
+    y = _special_bf16(rng, (rows, H))
+    ys = _special_bf16(rng, (T, H)) if shared else None
+    w = rng.uniform(0, 1, (T, K)).astype(np.float32)
+    kind = rng.random((T, K))
+    w[kind < 0.1] = 0.0
+    w[(kind >= 0.1) & (kind < 0.15)] = np.float32(3e-40)
+    w[(kind >= 0.15) & (kind < 0.2)] *= -1.0
+    w[(kind >= 0.2) & (kind < 0.22)] = np.float32(1e30)
+    w[(kind >= 0.22) & (kind < 0.225)] = np.inf
+    dest = rng.permutation(rows).astype(np.int32).reshape(T, K)
+    dest[rng.random((T, K)) < 0.05] = -1
+    cfg = moe.Config(T=T, H=H, E=max(K, 8), K=K, I=128)
+    dev = lambda a: None if a is None else torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(DEV)
+    bf = lambda a: None if a is None else dev(a).view(torch.bfloat16)
+    out = moe.combine(cfg, bf(y), dev(w), dev(dest), y_shared=bf(ys), order_invariant=True)
+    ref = oracle.combine_invariant(y, w, dest, ys, None)
+    got = bits(out)
+    nan_ref = (ref & 0x7fff) > 0x7f80
+    nan_got = (got & 0x7fff) > 0x7f80
+    assert np.array_equal(nan_got, nan_ref)
+    assert np.array_equal(got[~nan_ref], ref[~nan_ref])
+    perm = np.argsort(rng.random((T, K)), axis=1)
+    out2 = moe.combine(cfg, bf(y), dev(np.take_along_axis(w, perm, 1)),
+                       dev(np.take_along_axis(dest, perm, 1)), y_shared=bf(ys),
+                       order_invariant=True)
+    assert np.array_equal(bits(out2), got)
