@@ -101,15 +101,23 @@ __device__ __forceinline__ float elementwise_score(float l, int score_fn)
 // by comparisons and a butterfly, e = exp_rl(l - m), the 32-lane tree sum (each lane's
 // experts in increasing order, then butterfly levels 16 .. 1), s = e / S; sigmoid and
 // sqrtsoftplus elementwise.
+// lane L's logits of one row (experts L, L+32, ...; 0 past E)
 template <int NE>
-__device__ __forceinline__ void contract_scores(const float* __restrict__ row, int E,
-                                                int score_fn, int lane, float (&s)[NE])
+__device__ __forceinline__ void load_row(const float* __restrict__ row, int E, int lane,
+                                         float (&s)[NE])
 {
 #pragma unroll
     for (int i = 0; i < NE; ++i) {
         const int e = lane + 32 * i;
         s[i] = (e < E) ? row[e] : 0.0f;
     }
+}
+
+// the scores of a row already loaded by load_row, in place
+template <int NE>
+__device__ __forceinline__ void contract_scores_of(int E, int score_fn, int lane,
+                                                   float (&s)[NE])
+{
     if (score_fn != MOE_SOFTMAX) {
 #pragma unroll
         for (int i = 0; i < NE; ++i) s[i] = elementwise_score(s[i], score_fn);
@@ -137,6 +145,14 @@ __device__ __forceinline__ void contract_scores(const float* __restrict__ row, i
         part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, off));
 #pragma unroll
     for (int i = 0; i < NE; ++i) s[i] = __fdiv_rn(s[i], part);
+}
+
+template <int NE>
+__device__ __forceinline__ void contract_scores(const float* __restrict__ row, int E,
+                                                int score_fn, int lane, float (&s)[NE])
+{
+    load_row<NE>(row, E, lane, s);
+    contract_scores_of<NE>(E, score_fn, lane, s);
 }
 
 // order-preserving 32-bit image of a choice: -0 == +0, NaN below every number

@@ -6,8 +6,9 @@
 //
 // Deterministic without float atomics: block b owns 64 consecutive tokens, warp w of it 8
 // of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
-// ...); the 8 warp partials are added in warp order, then the block partials in block order
-// by the finishing kernel, and aux is a fixed tree over the experts. The result depends on
+// ...); the 8 warp partials are added in warp order, then the block partials by the
+// finishing kernel in a fixed order (contiguous slices of blocks in block order, then the
+// slices in order), and aux is a fixed tree over the experts. The result depends on
 // T (a batch statistic), never on scheduling.
 #include "route_math.cuh"
 
@@ -34,13 +35,32 @@ __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __re
     for (int i = 0; i < NE; ++i) acc[i] = 0.0f;
     int n_kept = 0;
     const int64_t t0 = (int64_t)blockIdx.x * kTokPerBlock + (int64_t)wid * kTokPerWarp;
+    // up to 128 experts the warp's rows are loaded before the first is scored (independent
+    // loads in flight); the tokens are still added in order
+    constexpr int kPre = NE <= 4 ? kTokPerWarp : 1;
+    float pre[kPre][NE];
+    if constexpr (kPre > 1) {
+#pragma unroll
+        for (int r = 0; r < kPre; ++r) {
+            const int64_t t = t0 + r;
+            const bool live = t < T && (mask == nullptr || mask[t] != 0);
+            if (live) load_row<NE>(logits + t * E, E, lane, pre[r]);
+        }
+    }
+#pragma unroll
     for (int r = 0; r < kTokPerWarp; ++r) {
         const int64_t t = t0 + r;
         if (t >= T) break;
         if (mask != nullptr && mask[t] == 0) continue;
         ++n_kept;
         float s[NE];
-        contract_scores<NE>(logits + t * E, E, score_fn, lane, s);
+        if constexpr (kPre > 1) {
+#pragma unroll
+            for (int i = 0; i < NE; ++i) s[i] = pre[r][i];
+        } else {
+            load_row<NE>(logits + t * E, E, lane, s);
+        }
+        contract_scores_of<NE>(E, score_fn, lane, s);
         // L1 normalisation over the experts with the same 32-lane tree
         float l1 = 0.0f;
 #pragma unroll
@@ -72,7 +92,10 @@ __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __re
     }
 }
 
-// one block of 1024 threads, thread e owns expert e
+// One block of 1024 threads. The block partials of expert e are summed in S contiguous
+// slices of blocks (S = the largest power of two <= 8 with S * E <= 1024; thread
+// s * E + e sums slice s in block order), then the S slice sums in slice order by thread e;
+// the kept-token count is an integer sum.
 __global__ void __launch_bounds__(1024) stats_finish_kernel(const float* __restrict__ partial,
                                                             const int32_t* __restrict__ kept,
                                                             int nblocks, int E,
@@ -83,13 +106,42 @@ __global__ void __launch_bounds__(1024) stats_finish_kernel(const float* __restr
 {
     pdl_wait();
     __shared__ float wsum[32];
-    const int e = threadIdx.x, lane = e & 31, wid = e >> 5;
-    int64_t n = 0;
-    for (int b = 0; b < nblocks; ++b) n += kept[b];
+    __shared__ float slice_sum[1024];
+    __shared__ unsigned long long n_kept;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) n_kept = 0ull;
+    __syncthreads();
+    {
+        unsigned long long k = 0ull;
+        for (int b = tid; b < nblocks; b += blockDim.x) k += (unsigned long long)kept[b];
+        if (k != 0ull) atomicAdd(&n_kept, k);
+    }
+    int S = 1;
+    while (S < 8 && 2 * S * E <= (int)blockDim.x) S *= 2;
+    const int per = (nblocks + S - 1) / S;
+    if (tid < S * E) {
+        const int e = tid % E, sl = tid / E;
+        const int b0 = sl * per, b1 = min(nblocks, b0 + per);
+        float v = 0.0f;
+        int b = b0;
+        // eight blocks' values loaded at a time (independent loads in flight), added in order
+        for (; b + 8 <= b1; b += 8) {
+            float pv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) pv[q] = partial[(int64_t)(b + q) * E + e];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v = __fadd_rn(v, pv[q]);
+        }
+        for (; b < b1; ++b) v = __fadd_rn(v, partial[(int64_t)b * E + e]);
+        slice_sum[tid] = v;
+    }
+    __syncthreads();
+    const int64_t n = (int64_t)n_kept;
+    const int e = tid;
     float term = 0.0f;
     if (e < E) {
-        float v = 0.0f;
-        for (int b = 0; b < nblocks; ++b) v = __fadd_rn(v, partial[(int64_t)b * E + e]);
+        float v = slice_sum[e];
+        for (int sl = 1; sl < S; ++sl) v = __fadd_rn(v, slice_sum[sl * E + e]);
         const int32_t c = offsets[e + 1] - offsets[e];
         counts[e] = c;
         const float nf = (float)n;

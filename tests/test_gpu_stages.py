@@ -146,8 +146,11 @@ def test_route_golden_two_token(golden):
 
 @pytest.mark.parametrize("T,K,E", [(1, 1, 8), (64, 2, 8), (3001, 8, 128), (8192, 1, 8),
                                    (2048, 6, 256), (777, 16, 1024), (20000, 8, 128),
-                                   (40000, 8, 256), (5000, 16, 1024)])
+                                   (40000, 8, 256), (5000, 16, 1024), (32768, 8, 128),
+                                   (16385, 16, 64)])
 def test_permute_bit_exact(T, K, E):
+    """Counting sort, bit-exact against the oracle: skewed loads, empty experts, padding and a
+    bad id, from one assignment to 320000 (157 blocks of 2048), E up to 1024."""
     rng = np.random.default_rng(T + K + E)
     # skewed expert choice (uneven loads, some experts empty), masked tokens, bad ids
     p = rng.dirichlet(np.full(E, 0.3))
