@@ -196,6 +196,13 @@ cudaError_t gate_up(const uint16_t* a, int64_t a_rows, const int32_t* gather, in
     p.ldo = I;
     p.status = status;
     if (gather != nullptr) return launch_tc_gemm_pair(p, st);
+    if (offsets != nullptr && grouped_rows <= 128) {
+        // no expert can have more than 128 rows (decode-sized batches): the one-SM kernel
+        // alone, its tiles dealt by CTA index (the pair launch would find no tile)
+        p.side_sms = 0;
+        p.tail_ctr = nullptr;
+        return launch_tc_gemm_tail(p, st);
+    }
     // experts of more than 128 rows on CTA pairs (the last tile padded), smaller ones on
     // single SMs: no expert's weights are read by both kernels (the same bits either way).
     // Where small experts are common (about 64 to 512 rows per expert on average) the two
