@@ -425,8 +425,6 @@ cudaError_t launch_tail_variant(const GemmProblem& p, cudaStream_t st)
     // CTA index: its side SMs. With the counter: a CTA per SM, the first side_sms of them
     // running beside the pair tiles and the rest taking what is left as pair CTAs finish.
     int64_t grid = (int64_t)groups * a.n_tiles;
-    // no more groups with rows than rows
-    if (p.offsets && rows_total >= 0 && rows_total < groups) grid = rows_total * a.n_tiles;
     if (a.side && a.tile_ctr == nullptr && grid > p.side_sms) grid = p.side_sms;
     if (grid > num_sms()) grid = num_sms();
     if (grid < 1) grid = 1;
