@@ -5,19 +5,21 @@
 // with s the unbiased scores of the routing contract (softmax, sigmoid or sqrtsoftplus).
 //
 // Deterministic without float atomics: block b owns 64 consecutive tokens, warp w of it 8
-// of them, summed in token order into per-lane registers (lane L holds experts L, L+32,
-// ...); the 8 warp partials are added in warp order, then the block partials by the
-// finishing kernel in a fixed order (contiguous slices of blocks in block order, then the
-// slices in order), and aux is a fixed tree over the experts. The result depends on
-// T (a batch statistic), never on scheduling.
+// of them (32 and 4 above 128 experts), summed in token order into per-lane registers (lane
+// L holds experts L, L+32, ...); the 8 warp partials are added in warp order, then the block
+// partials by the finishing kernel in a fixed order (contiguous slices of blocks in block
+// order, then the slices in order), and aux is a fixed tree over the experts. The result
+// depends on T and E (a batch statistic), never on scheduling.
 #include "route_math.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kTokPerBlock = 64;
+// tokens per warp: 8 up to 128 experts (their rows are loaded ahead, so a warp has enough
+// loads in flight), 4 above (more warps; measured 36.6 -> 26.2 us at 256 experts, T = 8192,
+// and slower at 128 experts: 25.1 -> 28.9 us at T = 16384)
+__host__ __device__ constexpr int tok_per_warp(int ne) { return ne <= 4 ? 8 : 4; }
 constexpr int kWarps = 8;
-constexpr int kTokPerWarp = kTokPerBlock / kWarps;
 
 template <int NE>
 __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __restrict__ logits,
@@ -34,7 +36,8 @@ __global__ void __launch_bounds__(kWarps * 32) prob_sum_kernel(const float* __re
 #pragma unroll
     for (int i = 0; i < NE; ++i) acc[i] = 0.0f;
     int n_kept = 0;
-    const int64_t t0 = (int64_t)blockIdx.x * kTokPerBlock + (int64_t)wid * kTokPerWarp;
+    constexpr int kTokPerWarp = tok_per_warp(NE);
+    const int64_t t0 = (int64_t)blockIdx.x * (kWarps * kTokPerWarp) + (int64_t)wid * kTokPerWarp;
     // up to 128 experts the warp's rows are loaded before the first is scored (independent
     // loads in flight); the tokens are still added in order
     constexpr int kPre = NE <= 4 ? kTokPerWarp : 1;
@@ -181,7 +184,8 @@ cudaError_t launch_ne(const moe_cfg& c, const float* logits, const uint8_t* mask
 
 size_t stats_ws_bytes(const moe_cfg& c)
 {
-    const int64_t nb = ((int64_t)c.T + kTokPerBlock - 1) / kTokPerBlock;
+    const int tpb = kWarps * tok_per_warp((c.E + 31) / 32);
+    const int64_t nb = ((int64_t)c.T + tpb - 1) / tpb;
     const int64_t n = nb > 0 ? nb : 1;
     return (size_t)n * c.E * sizeof(float) + (size_t)n * sizeof(int32_t) + 256;
 }
@@ -190,7 +194,8 @@ cudaError_t launch_router_stats(const moe_cfg& c, const float* logits, const uin
                                 const int32_t* offsets, int32_t* counts, float* mean_prob,
                                 float* aux, void* ws, cudaStream_t st)
 {
-    const int nb = (int)(((int64_t)c.T + kTokPerBlock - 1) / kTokPerBlock);
+    const int tpb = kWarps * tok_per_warp((c.E + 31) / 32);
+    const int nb = (int)(((int64_t)c.T + tpb - 1) / tpb);
     float* partial = static_cast<float*>(ws);
     int32_t* kept = reinterpret_cast<int32_t*>(
         static_cast<char*>(ws) + (size_t)(nb > 0 ? nb : 1) * c.E * sizeof(float));
